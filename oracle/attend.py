@@ -12,7 +12,8 @@ A2  tokens appended after the selection snapshot, [tail_begin, T_b), are
     always attended in addition to the selected set (a consequence of the
     selection running one step ahead; the pages do not discuss it).
 A3  logits q . k_j / sqrt(d), softmax over the attended set, output
-    sum_j p_j v_j; lse = log sum_j exp(logit_j) (natural log).
+    sum_j p_j v_j; lse = log sum_j exp(logit_j) (natural log).  An empty set
+    (an empty sum) gives output 0 and lse = -inf.
 
 Pins (tests/test_oracle_attend.py): with every token selected the result is
 dense attention, checked against torch's scaled_dot_product_attention run in
@@ -31,6 +32,8 @@ def attend_set(q: np.ndarray, K: np.ndarray, V: np.ndarray, S: np.ndarray):
     """``q [G, d]``, ``K, V [T, d]``, attended token set ``S`` -> (``o [G, d]``, ``lse [G]``)."""
     q = np.asarray(q, dtype=np.float64)
     S = np.unique(np.asarray(S, dtype=np.int64))
+    if S.size == 0:
+        return np.zeros_like(q), np.full(q.shape[0], -np.inf)
     Ks = np.asarray(K[S], dtype=np.float64)
     Vs = np.asarray(V[S], dtype=np.float64)
     logits = q @ Ks.T / math.sqrt(q.shape[-1])          # [G, |S|]

@@ -76,3 +76,9 @@ def test_tail_tokens_are_added_to_the_selection():
     out, _ = A.sparse_attend(q, keys, vals, idx, cnt, tail_begin=[16])
     ref, _ = A.attend_set(q[0], keys[0][0], vals[0][0], np.array([2, 5, 16, 17, 18, 19]))
     assert np.allclose(out[0], ref, rtol=1e-14, atol=1e-14)
+
+
+def test_empty_set_is_an_empty_sum():
+    q = RNG.standard_normal((2, 8))
+    o, lse = A.attend_set(q, RNG.standard_normal((5, 8)), RNG.standard_normal((5, 8)), np.array([], dtype=np.int64))
+    assert np.array_equal(o, np.zeros((2, 8))) and np.all(lse == -np.inf)
