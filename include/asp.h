@@ -1,0 +1,288 @@
+/*
+ * asp.h -- C ABI of libasp: predicted-query token-level sparse decode attention
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The method (AsyncSpade, "Efficient Test-Time Scaling with Asynchronous Sparse
+ * Decoding") removes KV selection from the decoding loop's critical path: while
+ * step t attends over the tokens chosen for it, the selection for step t+1 is
+ * made from a *predicted* query (abstract, components (1) and (2); research-map
+ * summary, "Approach").  The pages print no API; these calls follow that problem
+ * statement:
+ *
+ *   asp_predict_query   step 1: next query from the last W queries (ridge + softmax
+ *                       coefficients + multi-window average pooling)
+ *   asp_score_keys      step 2: every cached key of a KV head scored with its
+ *                       group's predicted queries
+ *   asp_select_topk     step 3: the C best tokens per (sequence, KV head)
+ *   asp_sparse_attend   step 4: single-token attention over the selected K/V only,
+ *                       with the true current query
+ *   asp_decode_step     steps 1-4 for one decode step: attention of step t on one
+ *                       stream, the selection for step t+1 on a side stream
+ *   asp_quest_*         the page-level comparison path (min/max page metadata)
+ *
+ * Conventions for every call:
+ *   - Pointers named as device memory must be device memory of the current CUDA
+ *     device; they stay owned by the caller.  The library never allocates device
+ *     or host memory for these calls and keeps no host-side state between calls.
+ *   - Work is enqueued asynchronously on the stream(s) given; a call returns once
+ *     the work is enqueued.  Stream and event handles are plain CUDA runtime
+ *     handles (cudaStream_t / cudaEvent_t); NULL stream means the legacy default
+ *     stream.
+ *   - Arguments are validated on the host before anything is enqueued.  On an
+ *     invalid argument the call returns a status other than ASP_OK and enqueues
+ *     nothing.  A failed launch returns ASP_ERR_CUDA.  No C++ exception crosses
+ *     this boundary.
+ *   - Device-side checks never trap: an out-of-range token index or page id is
+ *     skipped, a bounded wait that runs out stops its warp, and either event sets
+ *     the library's device status word, read with asp_device_status().
+ *   - Layouts are row-major; "[a, b, c]" lists dimensions outermost first.
+ *   - GQA: query head hq belongs to KV head hq / G, G = n_q_heads / n_kv_heads.
+ */
+#ifndef ASP_H_
+#define ASP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ASP_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define ASP_API __attribute__((visibility("default")))
+#else
+#define ASP_API
+#endif
+
+/* ABI-compatible with cudaStream_t / cudaEvent_t. */
+typedef struct CUstream_st* asp_stream_t;
+typedef struct CUevent_st* asp_event_t;
+
+typedef enum {
+  ASP_OK = 0,
+  ASP_ERR_INVALID_ARG = 1,  /* null pointer, bad size or inconsistent shapes */
+  ASP_ERR_UNSUPPORTED = 2,  /* valid but not built: head_dim, group size, dtype combination */
+  ASP_ERR_WORKSPACE = 3,    /* workspace missing or smaller than the matching *_workspace_bytes() */
+  ASP_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  ASP_ERR_TIMEOUT = 5,      /* asp_wait_selection: the event did not complete in time */
+  ASP_ERR_DEVICE = 6        /* asp_device_status: a kernel recorded a device-side fault */
+} asp_status;
+
+typedef enum { ASP_F32 = 0, ASP_BF16 = 1 } asp_dtype;
+
+/* How the ridge coefficients of one window become weights (softmax is the
+ * method's "softmax-normalized" reading; RAW keeps the coefficients). */
+typedef enum { ASP_COEF_SOFTMAX = 0, ASP_COEF_RAW = 1 } asp_coef_mode;
+
+/* Device status word bits (asp_device_status). */
+#define ASP_DEV_BAD_INDEX  0x1   /* a selected index outside [0, T_b) was skipped */
+#define ASP_DEV_BAD_PAGE   0x2   /* a page-table entry outside [0, n_pages) was skipped */
+#define ASP_DEV_WAIT_LIMIT 0x4   /* a bounded shared-memory barrier wait ran out */
+#define ASP_DEV_TAIL_LIMIT 0x8   /* a tail longer than max_tail was truncated */
+
+/* The KV cache of one layer.
+ *   page_size == 0: k, v are [batch, n_kv_heads, t_max, head_dim] (contiguous).
+ *   page_size  > 0: k, v are [n_pages, n_kv_heads, page_size, head_dim]; token j of
+ *                   sequence b lives in page page_table[b * max_pages + j / page_size]
+ *                   at row j % page_size.  page_size must be a multiple of 16, at most 256.
+ * seq_lens[b] = T_b, the number of valid tokens of sequence b (device int32 [batch],
+ * 0 <= T_b <= t_max; larger values are clamped to t_max).  NULL means T_b = t_max.
+ * Paged caches require seq_lens and page_table (device int32 [batch, max_pages]),
+ * t_max <= max_pages * page_size.  k, v must be 16-byte aligned. */
+typedef struct {
+  int batch;
+  int n_kv_heads;
+  int head_dim;          /* 64 or 128 */
+  int t_max;             /* token capacity of a sequence; row stride of score buffers */
+  asp_dtype kv_dtype;    /* ASP_F32 or ASP_BF16 */
+  const void* k;
+  const void* v;
+  int page_size;
+  const int32_t* page_table;
+  int max_pages;
+  int n_pages;           /* physical pages in the pool (paged only) */
+  const int32_t* seq_lens;
+} asp_kv;
+
+/* Predictor configuration (host memory). */
+typedef struct {
+  int W;                 /* lags; the history holds W + 1 vectors, 1 <= W <= 32 */
+  const int* windows;    /* pooling windows, each in [1, W], 1 to 8 of them */
+  int n_windows;
+  float lambda;          /* ridge parameter, > 0, added to the Gram diagonal unscaled */
+  asp_coef_mode coef;
+} asp_pred_cfg;
+
+/* ---------------------------------------------------------------------------
+ * Step 1 -- predicted query.
+ * Source: abstract, component (1) (a light-weight temporal-regressive module
+ * predicts the next query from a short window of recent queries); research-map
+ * summary, "Approach" (softmax-normalized ridge regression with multi-window
+ * average pooling); reproduction card, claim C5 (one-step-ahead fit, 16-query
+ * window).  For each query head and each window w: ridge-fit q_t on the lags
+ * q_{t-w}..q_{t-1} over the head_dim channels, a = (X X^T + lambda I)^-1 X q_t,
+ * turn a into weights (softmax or raw), apply weight i to q_{t-w+i}; average
+ * the window predictions.  Gram, Cholesky solve and weights run in fp64.
+ *
+ * qhist : device fp32 ring [batch, n_q_heads, W+1, head_dim].  Slot
+ *         (ring_start + s) % (W+1) holds the s-th oldest vector (s = 0..W).
+ * q_new : NULL, or device [batch, n_q_heads, head_dim] of q_new_dtype.  When given,
+ *         the oldest slot (ring_start) is first overwritten with q_new (as fp32),
+ *         so the window becomes slots ring_start+1 .. ring_start+W+1; the caller
+ *         then advances its ring_start by one.  Without it qhist is only read.
+ * qpred : device fp32 [batch, n_q_heads, head_dim], written.
+ * Errors: ASP_ERR_INVALID_ARG (null pointers, sizes <= 0, windows outside [1, W],
+ * lambda <= 0, ring_start outside [0, W]); ASP_ERR_UNSUPPORTED (head_dim not 64/128,
+ * W > 32). */
+ASP_API asp_status asp_predict_query(float* qhist, int ring_start, const void* q_new, asp_dtype q_new_dtype,
+                             int batch, int n_q_heads, int head_dim, const asp_pred_cfg* cfg,
+                             float* qpred, asp_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Step 2 -- score every cached key.
+ * Source: abstract (query-aware, token-level KV selection replacing page
+ * filtering); research-map summary, "Key results" (Qwen3 GQA models).
+ * scores[b, h, j] = max over the G query heads g of KV head h of
+ *                   (qpred[b, h*G + g, :] . k[b, h, j, :]) / sqrt(head_dim),  j < T_b.
+ * Entries j >= T_b of a row are not written.  fp32 arithmetic.
+ * qpred  : device fp32 [batch, n_q_heads, head_dim].
+ * scores : device fp32 [batch, n_kv_heads, t_max], written.
+ * Errors: ASP_ERR_INVALID_ARG; ASP_ERR_UNSUPPORTED (G not in {1,2,4,8}, head_dim
+ * not 64/128, batch > 8192). */
+ASP_API asp_status asp_score_keys(const float* qpred, int n_q_heads, const asp_kv* kv, float* scores,
+                          asp_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Step 3 -- top-C token selection.
+ * Source: research-map summary, "Key results" (2k selected tokens); reproduction
+ * card, "Key finding" (C = 2k tokens).  Per row (b, h): the C largest of
+ * scores[b, h, 0:T_b] under IEEE order (-0.0 == +0.0; +-inf allowed; NaN is not
+ * allowed), ties at the threshold going to the lowest token index.  The chosen
+ * indices are written in ascending order; count = min(C, T_b); entries past count
+ * are -1.
+ * scores   : device fp32 [batch, n_kv_heads, t_max] (only j < T_b is read).
+ * seq_lens : device int32 [batch] or NULL (T_b = t_max).
+ * idx      : device int32 [batch, n_kv_heads, C], written.
+ * count    : device int32 [batch, n_kv_heads], written.
+ * Errors: ASP_ERR_INVALID_ARG; ASP_ERR_UNSUPPORTED (t_max > 262144). */
+ASP_API asp_status asp_select_topk(const float* scores, const int32_t* seq_lens, int batch, int n_kv_heads,
+                           int t_max, int C, int32_t* idx, int32_t* count, asp_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Step 4 -- single-token attention over the selected tokens.
+ * Source: abstract (attention over the selected KV; selection decoupled from the
+ * decoding loop); reproduction card, "Key finding" (both methods attend to the
+ * same 2k tokens).  For query head hq of KV head h, with S = {idx[b,h,0:count]} u
+ * [tail_begin[b], T_b):
+ *   out[b, hq] = sum_{j in S} softmax_j(q[b,hq] . k_j / sqrt(d)) v_j,
+ *   lse[b, hq] = ln sum_{j in S} exp(q[b,hq] . k_j / sqrt(d)).
+ * The query is the true current query.  Selected indices >= tail_begin[b] are
+ * covered by the tail and skipped; indices outside [0, T_b) are skipped and flagged.
+ * An empty S gives out = 0 and lse = -inf.  Split-K over S with a log-sum-exp merge;
+ * fp32 accumulation.
+ * q          : device [batch, n_q_heads, head_dim] of q_dtype (bf16 or fp32).
+ * idx, count : as written by asp_select_topk (idx row stride C).
+ * tail_begin : device int32 [batch] or NULL (no tail); max_tail bounds T_b - tail_begin
+ *              (longer tails are truncated and flagged).  max_tail = t_max with
+ *              tail_begin = 0 and count = 0 gives dense attention.
+ * out        : device [batch, n_q_heads, head_dim] in kv_dtype, written.
+ * lse        : device fp32 [batch, n_q_heads] or NULL.
+ * workspace  : device scratch of at least asp_attend_workspace_bytes(...) bytes
+ *              (any alignment of 256 bytes); contents need no initialisation.
+ * Errors: ASP_ERR_INVALID_ARG; ASP_ERR_UNSUPPORTED; ASP_ERR_WORKSPACE. */
+ASP_API asp_status asp_sparse_attend(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv,
+                             const int32_t* idx, const int32_t* count, int C,
+                             const int32_t* tail_begin, int max_tail,
+                             void* out, float* lse, void* workspace, size_t workspace_bytes,
+                             asp_stream_t stream);
+
+/* Bytes of workspace asp_sparse_attend needs for these sizes (a pure function of
+ * its arguments; 0 for invalid sizes). */
+ASP_API size_t asp_attend_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C,
+                                  int max_tail);
+
+/* ---------------------------------------------------------------------------
+ * One asynchronous decode step (steps 1-4).
+ * Source: abstract, component (2) (KV selection decoupled from the decoding loop
+ * and overlapped with the forward computation).  On one GPU the two ranks of the
+ * pages become two streams:
+ *   s_main : waits for ev_sel_done (the previous step's selection, i.e. idx_cur),
+ *            then attends q_t over idx_cur/count_cur (+ tail) -> out, lse.
+ *   s_side : waits for ev_fork (recorded on s_main at entry), pushes q_t into the
+ *            ring, predicts qpred, scores every key, selects idx_next/count_next,
+ *            then records ev_sel_done.
+ * The caller swaps idx_cur/idx_next (and count_*) between steps, advances
+ * ring_start by one, and must not reuse q_t, qpred, scores or idx_next before
+ * ev_sel_done completes.  timing: NULL, or 8 events recorded around the kernels
+ * (begin/end of predict, score, select on s_side; attend on s_main) for profiling. */
+typedef struct {
+  const void* q_t;              /* device [batch, n_q_heads, head_dim] */
+  asp_dtype q_dtype;
+  int n_q_heads;
+  float* qhist;                 /* ring, see asp_predict_query */
+  int ring_start;
+  const asp_pred_cfg* pred;
+  const asp_kv* kv;
+  int C;
+  const int32_t* idx_cur;       /* [batch, n_kv_heads, C] */
+  const int32_t* count_cur;     /* [batch, n_kv_heads] */
+  const int32_t* tail_begin;    /* [batch] or NULL */
+  int max_tail;
+  float* qpred;                 /* [batch, n_q_heads, head_dim] scratch */
+  float* scores;                /* [batch, n_kv_heads, t_max] scratch */
+  int32_t* idx_next;            /* [batch, n_kv_heads, C] */
+  int32_t* count_next;          /* [batch, n_kv_heads] */
+  void* out;                    /* [batch, n_q_heads, head_dim] kv dtype */
+  float* lse;                   /* [batch, n_q_heads] or NULL */
+  void* workspace;
+  size_t workspace_bytes;
+  asp_stream_t s_main;
+  asp_stream_t s_side;
+  asp_event_t ev_fork;
+  asp_event_t ev_sel_done;
+  asp_event_t* timing;          /* NULL or asp_event_t[8] */
+} asp_decode_args;
+
+ASP_API asp_status asp_decode_step(const asp_decode_args* args);
+
+/* Host wait for a selection with a time limit (polls the event; never blocks past
+ * timeout_us).  Returns ASP_OK, ASP_ERR_TIMEOUT or ASP_ERR_CUDA. */
+ASP_API asp_status asp_wait_selection(asp_event_t ev_sel_done, long timeout_us);
+
+/* ---------------------------------------------------------------------------
+ * Page-level comparison path (Quest-style).
+ * Source: abstract and research-map summary, "Problem" (query-aware page-level
+ * filtering that waits for the current query); reproduction card, "Key finding"
+ * (its page-scan term 2 q h T/P).  Pages of quest_page tokens (a multiple of 16;
+ * for a paged cache it must equal kv->page_size).
+ * meta : device [batch, n_kv_heads, ceil(t_max / quest_page), 2, head_dim] in kv_dtype:
+ *        per page and channel the minimum (index 0) and maximum (index 1) key value
+ *        over the page's valid tokens. */
+ASP_API asp_status asp_quest_build_meta(const asp_kv* kv, int quest_page, void* meta, asp_stream_t stream);
+
+/* Page score u_p = max over the group's query heads of
+ * sum_c max(q_c kmin_c, q_c kmax_c) / sqrt(d) with the current query q; the
+ * ceil(C / quest_page) best pages (lowest page index on ties) are kept and their
+ * valid tokens written ascending to idx [batch, n_kv_heads, ceil(C/quest_page)*quest_page]
+ * (-1 padded), count [batch, n_kv_heads].
+ * page_scores : device fp32 scratch [batch, n_kv_heads, ceil(t_max / quest_page)]. */
+ASP_API asp_status asp_quest_select(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv,
+                            const void* meta, int quest_page, int C, float* page_scores,
+                            int32_t* idx, int32_t* count, asp_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Utilities. */
+
+/* Reads and clears the device status word (ASP_DEV_* bits) after synchronising
+ * `stream`.  Returns ASP_ERR_DEVICE when a bit was set, else ASP_OK/ASP_ERR_CUDA. */
+ASP_API asp_status asp_device_status(asp_stream_t stream, int32_t* bits_out);
+
+ASP_API const char* asp_status_string(asp_status status);
+ASP_API int asp_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ASP_H_ */

@@ -1,0 +1,341 @@
+// asp_api.cu -- the C ABI of libasp: host-side validation, dispatch to the
+// kernels, the two-stream decode step and small utilities.  Nothing here
+// allocates memory; every error is reported as an asp_status.
+#include <chrono>
+#include <cmath>
+#include <thread>
+
+#include "asp_common.cuh"
+#include "asp_internal.h"
+
+namespace asp {
+
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] <= 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) cache[dev] = n;
+  }
+  return cache[dev] > 0 ? cache[dev] : 148;
+}
+
+}  // namespace asp
+
+namespace {
+
+using asp::KvView;
+
+constexpr int kMaxGridY = 65535;
+constexpr int kMaxScoreBatch = 8192;   // the key scan keeps per-sequence offsets in shared memory
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool group_ok(int n_q_heads, int n_kv) {
+  if (n_kv <= 0 || n_q_heads <= 0 || n_q_heads % n_kv) return false;
+  const int g = n_q_heads / n_kv;
+  return g == 1 || g == 2 || g == 4 || g == 8;
+}
+
+// Validates a KV description; need_v: the call reads v too.
+asp_status check_kv(const asp_kv* kv, bool need_v) {
+  if (!kv) return ASP_ERR_INVALID_ARG;
+  if (kv->batch <= 0 || kv->n_kv_heads <= 0 || kv->t_max <= 0) return ASP_ERR_INVALID_ARG;
+  if (kv->kv_dtype != ASP_F32 && kv->kv_dtype != ASP_BF16) return ASP_ERR_INVALID_ARG;
+  if (kv->head_dim != 64 && kv->head_dim != 128) return ASP_ERR_UNSUPPORTED;
+  if (!kv->k || (need_v && !kv->v)) return ASP_ERR_INVALID_ARG;
+  if (!aligned16(kv->k) || (need_v && !aligned16(kv->v))) return ASP_ERR_INVALID_ARG;
+  if ((long)kv->batch * kv->n_kv_heads > kMaxGridY) return ASP_ERR_UNSUPPORTED;
+  if (kv->page_size < 0) return ASP_ERR_INVALID_ARG;
+  if (kv->page_size > 0) {
+    if (kv->page_size % 16 || kv->page_size > 256) return ASP_ERR_UNSUPPORTED;
+    if (!kv->page_table || !kv->seq_lens || kv->max_pages <= 0 || kv->n_pages <= 0) return ASP_ERR_INVALID_ARG;
+    if ((long)kv->max_pages * kv->page_size < kv->t_max) return ASP_ERR_INVALID_ARG;
+  }
+  return ASP_OK;
+}
+
+KvView view_of(const asp_kv* kv) {
+  KvView v;
+  v.k = kv->k;
+  v.v = kv->v;
+  v.kv_f32 = kv->kv_dtype == ASP_F32;
+  v.batch = kv->batch;
+  v.n_kv = kv->n_kv_heads;
+  v.head_dim = kv->head_dim;
+  v.t_max = kv->t_max;
+  v.page_size = kv->page_size;
+  v.max_pages = kv->page_size ? kv->max_pages : 0;
+  v.n_pages = kv->page_size ? kv->n_pages : 0;
+  v.page_table = kv->page_size ? kv->page_table : nullptr;
+  v.seq_lens = kv->seq_lens;
+  return v;
+}
+
+asp_status check_pred(const asp_pred_cfg* cfg, int ring_start) {
+  if (!cfg) return ASP_ERR_INVALID_ARG;
+  if (cfg->W < 1) return ASP_ERR_INVALID_ARG;
+  if (cfg->W > 32) return ASP_ERR_UNSUPPORTED;
+  if (!cfg->windows || cfg->n_windows < 1 || cfg->n_windows > 8) return ASP_ERR_INVALID_ARG;
+  for (int i = 0; i < cfg->n_windows; ++i)
+    if (cfg->windows[i] < 1 || cfg->windows[i] > cfg->W) return ASP_ERR_INVALID_ARG;
+  if (!(cfg->lambda > 0.0f) || !std::isfinite(cfg->lambda)) return ASP_ERR_INVALID_ARG;
+  if (cfg->coef != ASP_COEF_SOFTMAX && cfg->coef != ASP_COEF_RAW) return ASP_ERR_INVALID_ARG;
+  if (ring_start < 0 || ring_start > cfg->W) return ASP_ERR_INVALID_ARG;
+  return ASP_OK;
+}
+
+asp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ASP_OK : ASP_ERR_CUDA; }
+
+asp::PredictArgs predict_args(float* qhist, int ring_start, const void* q_new, asp_dtype q_new_dtype, int batch,
+                              int n_q_heads, int head_dim, const asp_pred_cfg* cfg, float* qpred) {
+  asp::PredictArgs a;
+  a.qhist = qhist;
+  a.ring_start = ring_start;
+  a.q_new = q_new;
+  a.q_new_f32 = q_new_dtype == ASP_F32;
+  a.n_heads = batch * n_q_heads;
+  a.W = cfg->W;
+  a.head_dim = head_dim;
+  a.n_win = cfg->n_windows;
+  a.wmax = 0;
+  for (int i = 0; i < 8; ++i) a.windows[i] = 0;
+  for (int i = 0; i < cfg->n_windows; ++i) {
+    a.windows[i] = cfg->windows[i];
+    if (cfg->windows[i] > a.wmax) a.wmax = cfg->windows[i];
+  }
+  a.lam = (double)cfg->lambda;
+  a.coef_raw = cfg->coef == ASP_COEF_RAW;
+  a.qpred = qpred;
+  return a;
+}
+
+asp_status check_attend(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv, const int32_t* idx,
+                        const int32_t* count, int C, const int32_t* tail_begin, int max_tail, void* out,
+                        void* workspace, size_t workspace_bytes, asp::AttendPlan* plan) {
+  asp_status st = check_kv(kv, true);
+  if (st != ASP_OK) return st;
+  if (!q || !out) return ASP_ERR_INVALID_ARG;
+  if (q_dtype != ASP_F32 && q_dtype != ASP_BF16) return ASP_ERR_INVALID_ARG;
+  if (n_q_heads <= 0 || n_q_heads % kv->n_kv_heads) return ASP_ERR_INVALID_ARG;
+  if (!group_ok(n_q_heads, kv->n_kv_heads)) return ASP_ERR_UNSUPPORTED;
+  if (C < 0 || (C > 0 && (!idx || !count))) return ASP_ERR_INVALID_ARG;
+  const int mt = tail_begin ? max_tail : 0;
+  if (mt < 0 || (long)C + mt < 1) return ASP_ERR_INVALID_ARG;
+  if ((long)C + mt > (1L << 30)) return ASP_ERR_UNSUPPORTED;
+  *plan = asp::attend_plan(kv->batch, n_q_heads, kv->n_kv_heads, kv->head_dim, C, mt);
+  if (plan->workspace_bytes) {
+    if (!workspace || workspace_bytes < plan->workspace_bytes) return ASP_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ASP_ERR_WORKSPACE;
+  }
+  return ASP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int asp_abi_version(void) { return ASP_ABI_VERSION; }
+
+const char* asp_status_string(asp_status s) {
+  switch (s) {
+    case ASP_OK: return "ok";
+    case ASP_ERR_INVALID_ARG: return "invalid argument";
+    case ASP_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ASP_ERR_WORKSPACE: return "workspace missing or too small";
+    case ASP_ERR_CUDA: return "CUDA error";
+    case ASP_ERR_TIMEOUT: return "timed out";
+    case ASP_ERR_DEVICE: return "device-side fault recorded";
+  }
+  return "unknown status";
+}
+
+asp_status asp_predict_query(float* qhist, int ring_start, const void* q_new, asp_dtype q_new_dtype, int batch,
+                             int n_q_heads, int head_dim, const asp_pred_cfg* cfg, float* qpred,
+                             asp_stream_t stream) {
+  if (!qhist || !qpred || batch <= 0 || n_q_heads <= 0) return ASP_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return ASP_ERR_UNSUPPORTED;
+  if (q_new && q_new_dtype != ASP_F32 && q_new_dtype != ASP_BF16) return ASP_ERR_INVALID_ARG;
+  if ((long)batch * n_q_heads > (1L << 28)) return ASP_ERR_UNSUPPORTED;
+  asp_status st = check_pred(cfg, ring_start);
+  if (st != ASP_OK) return st;
+  const asp::PredictArgs a = predict_args(qhist, ring_start, q_new, q_new_dtype, batch, n_q_heads, head_dim, cfg, qpred);
+  return cuda_status(asp::launch_predict(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+asp_status asp_score_keys(const float* qpred, int n_q_heads, const asp_kv* kv, float* scores, asp_stream_t stream) {
+  asp_status st = check_kv(kv, false);
+  if (st != ASP_OK) return st;
+  if (!qpred || !scores) return ASP_ERR_INVALID_ARG;
+  if (n_q_heads <= 0 || n_q_heads % kv->n_kv_heads) return ASP_ERR_INVALID_ARG;
+  if (!group_ok(n_q_heads, kv->n_kv_heads)) return ASP_ERR_UNSUPPORTED;
+  if (kv->batch > kMaxScoreBatch) return ASP_ERR_UNSUPPORTED;
+  return cuda_status(asp::launch_score(qpred, n_q_heads, view_of(kv), scores, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+asp_status asp_select_topk(const float* scores, const int32_t* seq_lens, int batch, int n_kv_heads, int t_max, int C,
+                           int32_t* idx, int32_t* count, asp_stream_t stream) {
+  if (!scores || !idx || !count || batch <= 0 || n_kv_heads <= 0 || t_max <= 0 || C <= 0) return ASP_ERR_INVALID_ARG;
+  if ((long)batch * n_kv_heads > kMaxGridY || !asp::select_supported(t_max, 1)) return ASP_ERR_UNSUPPORTED;
+  asp::SelectArgs a;
+  a.scores = scores;
+  a.row_stride = t_max;
+  a.seq_lens = seq_lens;
+  a.t_max = t_max;
+  a.rows_per_seq = n_kv_heads;
+  a.n_rows = batch * n_kv_heads;
+  a.c_units = C;
+  a.expand = 1;
+  a.idx = idx;
+  a.count = count;
+  return cuda_status(asp::launch_select(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t asp_attend_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail) {
+  if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || C < 0 || max_tail < 0 || (long)C + max_tail < 1) return 0;
+  if (head_dim != 64 && head_dim != 128) return 0;
+  return asp::attend_plan(batch, n_q_heads, n_kv_heads, head_dim, C, max_tail).workspace_bytes;
+}
+
+asp_status asp_sparse_attend(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv, const int32_t* idx,
+                             const int32_t* count, int C, const int32_t* tail_begin, int max_tail, void* out,
+                             float* lse, void* workspace, size_t workspace_bytes, asp_stream_t stream) {
+  asp::AttendPlan plan;
+  asp_status st = check_attend(q, q_dtype, n_q_heads, kv, idx, count, C, tail_begin, max_tail, out, workspace,
+                               workspace_bytes, &plan);
+  if (st != ASP_OK) return st;
+  return cuda_status(asp::launch_attend(q, q_dtype == ASP_F32, n_q_heads, view_of(kv), idx, count, C, tail_begin,
+                                        max_tail, out, lse, workspace, plan, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+asp_status asp_decode_step(const asp_decode_args* a) {
+  if (!a) return ASP_ERR_INVALID_ARG;
+  asp::AttendPlan plan;
+  asp_status st = check_attend(a->q_t, a->q_dtype, a->n_q_heads, a->kv, a->idx_cur, a->count_cur, a->C, a->tail_begin,
+                               a->max_tail, a->out, a->workspace, a->workspace_bytes, &plan);
+  if (st != ASP_OK) return st;
+  if (a->C < 1 || !a->qhist || !a->qpred || !a->scores || !a->idx_next || !a->count_next) return ASP_ERR_INVALID_ARG;
+  if (!a->ev_fork || !a->ev_sel_done) return ASP_ERR_INVALID_ARG;
+  st = check_pred(a->pred, a->ring_start);
+  if (st != ASP_OK) return st;
+  if (!asp::select_supported(a->kv->t_max, 1) || a->kv->batch > kMaxScoreBatch) return ASP_ERR_UNSUPPORTED;
+
+  cudaStream_t sm = reinterpret_cast<cudaStream_t>(a->s_main);
+  cudaStream_t ss = reinterpret_cast<cudaStream_t>(a->s_side);
+  cudaEvent_t fork = reinterpret_cast<cudaEvent_t>(a->ev_fork);
+  cudaEvent_t done = reinterpret_cast<cudaEvent_t>(a->ev_sel_done);
+  auto mark = [&](int i, cudaStream_t s) -> cudaError_t {
+    return a->timing ? cudaEventRecord(reinterpret_cast<cudaEvent_t>(a->timing[i]), s) : cudaSuccess;
+  };
+  const KvView kv = view_of(a->kv);
+  const int B = a->kv->batch;
+
+  cudaError_t e = cudaStreamWaitEvent(sm, done, 0);   // idx_cur: the previous step's selection
+  if (e == cudaSuccess) e = cudaEventRecord(fork, sm);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ss, fork, 0);
+  // side stream: selection for the next step
+  if (e == cudaSuccess) e = mark(0, ss);
+  if (e == cudaSuccess) {
+    const asp::PredictArgs pa = predict_args(a->qhist, a->ring_start, a->q_t, a->q_dtype, B, a->n_q_heads,
+                                             a->kv->head_dim, a->pred, a->qpred);
+    e = asp::launch_predict(pa, ss);
+  }
+  if (e == cudaSuccess) e = mark(1, ss);
+  if (e == cudaSuccess) e = mark(2, ss);
+  if (e == cudaSuccess) e = asp::launch_score(a->qpred, a->n_q_heads, kv, a->scores, ss);
+  if (e == cudaSuccess) e = mark(3, ss);
+  if (e == cudaSuccess) e = mark(4, ss);
+  if (e == cudaSuccess) {
+    asp::SelectArgs sa;
+    sa.scores = a->scores;
+    sa.row_stride = a->kv->t_max;
+    sa.seq_lens = a->kv->seq_lens;
+    sa.t_max = a->kv->t_max;
+    sa.rows_per_seq = a->kv->n_kv_heads;
+    sa.n_rows = B * a->kv->n_kv_heads;
+    sa.c_units = a->C;
+    sa.expand = 1;
+    sa.idx = a->idx_next;
+    sa.count = a->count_next;
+    e = asp::launch_select(sa, ss);
+  }
+  if (e == cudaSuccess) e = mark(5, ss);
+  if (e == cudaSuccess) e = cudaEventRecord(done, ss);
+  // main stream: attention of this step
+  if (e == cudaSuccess) e = mark(6, sm);
+  if (e == cudaSuccess)
+    e = asp::launch_attend(a->q_t, a->q_dtype == ASP_F32, a->n_q_heads, kv, a->idx_cur, a->count_cur, a->C,
+                           a->tail_begin, a->max_tail, a->out, a->lse, a->workspace, plan, sm);
+  if (e == cudaSuccess) e = mark(7, sm);
+  return cuda_status(e);
+}
+
+asp_status asp_wait_selection(asp_event_t ev_sel_done, long timeout_us) {
+  if (!ev_sel_done || timeout_us < 0) return ASP_ERR_INVALID_ARG;
+  const auto t0 = std::chrono::steady_clock::now();
+  for (;;) {
+    const cudaError_t e = cudaEventQuery(reinterpret_cast<cudaEvent_t>(ev_sel_done));
+    if (e == cudaSuccess) return ASP_OK;
+    if (e != cudaErrorNotReady) return ASP_ERR_CUDA;
+    const long waited = (long)std::chrono::duration_cast<std::chrono::microseconds>(
+                            std::chrono::steady_clock::now() - t0).count();
+    if (waited >= timeout_us) return ASP_ERR_TIMEOUT;
+    std::this_thread::sleep_for(std::chrono::microseconds(20));
+  }
+}
+
+asp_status asp_quest_build_meta(const asp_kv* kv, int quest_page, void* meta, asp_stream_t stream) {
+  asp_status st = check_kv(kv, false);
+  if (st != ASP_OK) return st;
+  if (!meta || quest_page <= 0) return ASP_ERR_INVALID_ARG;
+  if (quest_page % 16 || quest_page > 256) return ASP_ERR_UNSUPPORTED;
+  if (kv->page_size && kv->page_size != quest_page) return ASP_ERR_UNSUPPORTED;
+  return cuda_status(asp::launch_quest_meta(view_of(kv), quest_page, meta, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+asp_status asp_quest_select(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv, const void* meta,
+                            int quest_page, int C, float* page_scores, int32_t* idx, int32_t* count,
+                            asp_stream_t stream) {
+  asp_status st = check_kv(kv, false);
+  if (st != ASP_OK) return st;
+  if (!q || !meta || !page_scores || !idx || !count || C <= 0 || quest_page <= 0) return ASP_ERR_INVALID_ARG;
+  if (q_dtype != ASP_F32 && q_dtype != ASP_BF16) return ASP_ERR_INVALID_ARG;
+  if (n_q_heads <= 0 || n_q_heads % kv->n_kv_heads) return ASP_ERR_INVALID_ARG;
+  if (!group_ok(n_q_heads, kv->n_kv_heads)) return ASP_ERR_UNSUPPORTED;
+  if (quest_page % 16 || quest_page > 256) return ASP_ERR_UNSUPPORTED;
+  if (kv->page_size && kv->page_size != quest_page) return ASP_ERR_UNSUPPORTED;
+  if (!asp::select_supported(kv->t_max, quest_page)) return ASP_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = asp::launch_quest_score(q, q_dtype == ASP_F32, n_q_heads, view_of(kv), meta, quest_page,
+                                          page_scores, s);
+  if (e != cudaSuccess) return ASP_ERR_CUDA;
+  asp::SelectArgs sa;
+  sa.scores = page_scores;
+  sa.row_stride = (kv->t_max + quest_page - 1) / quest_page;
+  sa.seq_lens = kv->seq_lens;
+  sa.t_max = kv->t_max;
+  sa.rows_per_seq = kv->n_kv_heads;
+  sa.n_rows = kv->batch * kv->n_kv_heads;
+  sa.c_units = (C + quest_page - 1) / quest_page;
+  sa.expand = quest_page;
+  sa.idx = idx;
+  sa.count = count;
+  return cuda_status(asp::launch_select(sa, s));
+}
+
+asp_status asp_device_status(asp_stream_t stream, int32_t* bits_out) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = asp::read_status_predict(s, &v);
+  if (e == cudaSuccess) e = asp::read_status_score(s, &v);
+  if (e == cudaSuccess) e = asp::read_status_select(s, &v);
+  if (e == cudaSuccess) e = asp::read_status_attend(s, &v);
+  if (e == cudaSuccess) e = asp::read_status_quest(s, &v);
+  if (bits_out) *bits_out = v;
+  if (e != cudaSuccess) return ASP_ERR_CUDA;
+  return v ? ASP_ERR_DEVICE : ASP_OK;
+}
+
+}  // extern "C"

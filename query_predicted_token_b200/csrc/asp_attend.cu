@@ -1,0 +1,499 @@
+// asp_attend.cu -- step 4: single-token attention over the selected K/V rows.
+//
+// out[b, hq] = sum_{j in S} softmax_j(q . k_j / sqrt(d)) v_j over S = selected u tail.
+//
+// HBM-bound gather (each selected K and V row read once, 256 B for bf16 d=128).
+//  * grid = (splits, batch * n_kv): a CTA takes a contiguous slice of one KV head's
+//    attended rows and computes all G query heads of the group, so a row is read
+//    once for the whole group;
+//  * a warp gathers 16 rows per tile: each of its 32 lanes issues one 1-D bulk
+//    copy (TMA) of a K row (lanes 0-15) or a V row (lanes 16-31) into the warp's
+//    stage, all counted on one mbarrier; STAGES tiles are in flight per warp;
+//  * logits: 16-byte shared-memory vectors per lane, packed FMAs, warp
+//    reduce-scatter over the row's lanes; online softmax in base 2 (log2 e folded
+//    into the query scale); V accumulated in fp32 registers;
+//  * warps of a CTA merge through shared memory; with several splits the partial
+//    (max, sum, unnormalised output) go to the workspace and a small kernel does
+//    the log-sum-exp merge.
+#include <cfloat>
+
+#include "asp_common.cuh"
+#include "asp_internal.h"
+
+namespace asp {
+namespace {
+
+constexpr int kTile = 16;
+constexpr int kWarps = 4;
+constexpr int kTargetCtas = 592;   // 4 CTAs per SM of a 148-SM B200
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+struct AttParams {
+  const void* q;
+  int q_f32;
+  int n_q_heads;
+  const uint8_t* k;
+  const uint8_t* v;
+  int batch, n_kv, t_max, page_size, max_pages, n_pages;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  const int32_t* idx;
+  const int32_t* count;
+  int C;
+  const int32_t* tail_begin;
+  int max_tail;
+  int splits, rows_per_split;
+  float* part_o;
+  float* part_ml;
+  void* out;
+  float* lse;
+  float qscale;   // log2(e) / sqrt(d)
+};
+
+template <typename KT, int D, int G, int STAGES>
+__global__ void __launch_bounds__(kWarps * 32) attend_kernel(AttParams p) {
+  using E = Elem<KT>;
+  constexpr int ROW_BYTES = D * E::kBytes;
+  constexpr int LPR = ROW_BYTES / 16;
+  constexpr int RPS = 32 / LPR;
+  constexpr int CPL = E::kPerVec;
+  constexpr int NSTEP = kTile / RPS;
+  constexpr int TILE_BYTES = 2 * kTile * ROW_BYTES;
+  constexpr int SPP = (NSTEP * G <= 32) ? NSTEP : (32 / G);
+  constexpr int NPASS = NSTEP / SPP;
+  constexpr int NV = SPP * G;
+  constexpr int LPG = 32 / G;                         // lanes per head in the softmax stage
+  constexpr int RPL = (kTile + LPG - 1) / LPG;        // tile rows per lane in the softmax stage
+  static_assert(LPR >= 2 && 32 % LPR == 0 && NV <= 32 && G * LPR >= NV, "layout");
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* wbuf = smem + (size_t)warp * STAGES * TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kWarps * STAGES * TILE_BYTES) + warp * STAGES;
+  float* lg = reinterpret_cast<float*>(smem + (size_t)kWarps * STAGES * TILE_BYTES + kWarps * STAGES * 8) +
+              warp * (kTile * G + G);
+  float* cs = lg + kTile * G;
+
+  const int unit = blockIdx.y, split = blockIdx.x;
+  const int b = unit / p.n_kv, h = unit - b * p.n_kv;
+  int T = p.seq_lens ? p.seq_lens[b] : p.t_max;
+  T = T < 0 ? 0 : (T > p.t_max ? p.t_max : T);
+  int n_sel = p.count[unit];
+  n_sel = n_sel < 0 ? 0 : (n_sel > p.C ? p.C : n_sel);
+  int tb = T;
+  if (p.tail_begin) {
+    tb = p.tail_begin[b];
+    tb = tb < 0 ? 0 : (tb > T ? T : tb);
+  }
+  int tail = T - tb;
+  if (tail > p.max_tail) {
+    if (threadIdx.x == 0 && split == 0) flag_status(ASP_DEV_TAIL_LIMIT);
+    tail = p.max_tail;
+  }
+  const int n_rows = n_sel + tail;
+  const int r0 = split * p.rows_per_split;
+  const int r1 = min(n_rows, r0 + p.rows_per_split);
+  const int n_tiles = r1 > r0 ? (r1 - r0 + kTile - 1) / kTile : 0;
+  const int32_t* idx_row = p.idx + (size_t)unit * p.C;
+
+  if (lane == 0) {
+    for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+
+  // query of the G heads, scaled by log2(e)/sqrt(d)
+  float2 q2[G][CPL / 2];
+  {
+    const int c0 = (lane % LPR) * CPL;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const size_t off = (size_t)(b * p.n_q_heads + h * G + g) * D + c0;
+#pragma unroll
+      for (int c = 0; c < CPL / 2; ++c) {
+        float x0, x1;
+        if (p.q_f32) {
+          const float2 x = *reinterpret_cast<const float2*>(static_cast<const float*>(p.q) + off + 2 * c);
+          x0 = x.x;
+          x1 = x.y;
+        } else {
+          const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(p.q) + off + 2 * c);
+          x0 = __low2float(x);
+          x1 = __high2float(x);
+        }
+        q2[g][c] = make_float2(x0 * p.qscale, x1 * p.qscale);
+      }
+    }
+  }
+
+  // tile t of this warp covers rows r0 + (warp + t * kWarps) * kTile + [0, 16)
+  const int my_tiles = n_tiles > warp ? (n_tiles - warp + kWarps - 1) / kWarps : 0;
+
+  auto issue = [&](int t, int slot) -> uint32_t {
+    const int rr = lane & 15;
+    const bool isv = lane >= 16;
+    const int r = r0 + (warp + t * kWarps) * kTile + rr;
+    bool valid = r < r1;
+    int j = 0;
+    if (valid) {
+      if (r < n_sel) {
+        j = idx_row[r];
+        if (j < 0 || j >= T) {
+          valid = false;
+          if (!isv) flag_status(ASP_DEV_BAD_INDEX);
+        } else if (j >= tb) {
+          valid = false;   // covered by the tail
+        }
+      } else {
+        j = tb + (r - n_sel);
+      }
+    }
+    const uint8_t* src = nullptr;
+    if (valid) {
+      const uint8_t* base = isv ? p.v : p.k;
+      if (p.page_size == 0) {
+        src = base + ((size_t)unit * p.t_max + j) * ROW_BYTES;
+      } else {
+        const int page = p.page_table[(size_t)b * p.max_pages + j / p.page_size];
+        if (page < 0 || page >= p.n_pages) {
+          valid = false;
+          if (!isv) flag_status(ASP_DEV_BAD_PAGE);
+        } else {
+          src = base + (((size_t)page * p.n_kv + h) * p.page_size + (j % p.page_size)) * ROW_BYTES;
+        }
+      }
+    }
+    const uint32_t vm = __ballot_sync(0xffffffffu, valid) & 0xffffu;
+    uint8_t* dst = wbuf + slot * TILE_BYTES + (isv ? kTile * ROW_BYTES : 0) + rr * ROW_BYTES;
+    if (!valid) {
+#pragma unroll
+      for (int c = 0; c < ROW_BYTES / 16; ++c) reinterpret_cast<uint4*>(dst)[c] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)__popc(vm) * 2u * ROW_BYTES);
+    __syncwarp();
+    if (valid) bulk_g2s(dst, src, ROW_BYTES, &bars[slot]);
+    return vm;
+  };
+
+  float2 o2[G][CPL / 2];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int c = 0; c < CPL / 2; ++c) o2[g][c] = make_float2(0.f, 0.f);
+  float m_run = -INFINITY;   // running max (base 2) of head lane % G
+  float l_run = 0.f;         // this lane's share of the running sum of head lane % G
+
+  uint32_t vmask[STAGES];
+  int issued = 0;
+#pragma unroll 1
+  for (int s = 0; s < STAGES && s < my_tiles; ++s) {
+    vmask[s] = issue(s, s);
+    ++issued;
+  }
+
+  int consumed = 0;
+  bool ok = true;
+#pragma unroll 1
+  for (int t = 0; t < my_tiles; ++t) {
+    const int slot = t % STAGES;
+    ok = __all_sync(0xffffffffu, mbar_wait(&bars[slot], (uint32_t)(t / STAGES) & 1u));
+    if (!ok) break;
+    ++consumed;
+    const uint32_t vm = vmask[slot];
+    const uint8_t* kb = wbuf + slot * TILE_BYTES;
+    const uint8_t* vb = kb + kTile * ROW_BYTES;
+
+    // 1. logits (base 2) of the 16 rows x G heads -> lg[row][g]
+#pragma unroll
+    for (int pass = 0; pass < NPASS; ++pass) {
+      float vals[NV];
+#pragma unroll
+      for (int s = 0; s < SPP; ++s) {
+        const int row = (pass * SPP + s) * RPS + lane / LPR;
+        const uint4 v = *reinterpret_cast<const uint4*>(kb + row * ROW_BYTES + (lane % LPR) * 16);
+        float2 kf[CPL / 2];
+        E::unpack(v, kf);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float2 acc = __fmul2_rn(kf[0], q2[g][0]);
+#pragma unroll
+          for (int c = 1; c < CPL / 2; ++c) acc = __ffma2_rn(kf[c], q2[g][c], acc);
+          vals[s * G + g] = acc.x + acc.y;
+        }
+      }
+      ReduceScatter<NV, LPR / 2>::run(vals, lane);
+      const int l = lane % LPR;
+      if constexpr (NV >= LPR) {
+        constexpr int VPL = NV / LPR;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+          const int pidx = VPL * l + i;
+          const int row = (pass * SPP + pidx / G) * RPS + lane / LPR;
+          lg[row * G + pidx % G] = vals[i];
+        }
+      } else {
+        const int pidx = l / (LPR / NV);
+        const int row = (pass * SPP + pidx / G) * RPS + lane / LPR;
+        lg[row * G + pidx % G] = vals[0];
+      }
+    }
+    __syncwarp();
+
+    // 2. online softmax statistics; probabilities overwrite the logits
+    {
+      const int g = lane % G, rl = lane / G;
+      float x[RPL];
+      float mloc = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < RPL; ++k) {
+        const int row = rl + k * LPG;
+        x[k] = (row < kTile && ((vm >> row) & 1u)) ? lg[row * G + g] : -INFINITY;
+        mloc = fmaxf(mloc, x[k]);
+      }
+#pragma unroll
+      for (int o = G; o < 32; o <<= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+      const float m_new = fmaxf(m_run, mloc);
+      const float corr = (m_new == -INFINITY) ? 1.f : ex2(m_run - m_new);
+      float psum = 0.f;
+#pragma unroll
+      for (int k = 0; k < RPL; ++k) {
+        const int row = rl + k * LPG;
+        const float pr = (x[k] == -INFINITY) ? 0.f : ex2(x[k] - m_new);
+        if (row < kTile) lg[row * G + g] = pr;
+        psum += pr;
+      }
+      l_run = l_run * corr + psum;
+      m_run = m_new;
+      if (lane < G) cs[lane] = corr;
+    }
+    __syncwarp();
+
+    // 3. rescale and accumulate V
+    {
+      bool any = false;
+      float cr[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        cr[g] = cs[g];
+        any |= cr[g] != 1.f;
+      }
+      if (any) {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int c = 0; c < CPL / 2; ++c) o2[g][c] = __fmul2_rn(o2[g][c], make_float2(cr[g], cr[g]));
+      }
+#pragma unroll
+      for (int s = 0; s < NSTEP; ++s) {
+        const int row = s * RPS + lane / LPR;
+        const uint4 v = *reinterpret_cast<const uint4*>(vb + row * ROW_BYTES + (lane % LPR) * 16);
+        float2 vf[CPL / 2];
+        E::unpack(v, vf);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float pr = lg[row * G + g];
+          const float2 pp = make_float2(pr, pr);
+#pragma unroll
+          for (int c = 0; c < CPL / 2; ++c) o2[g][c] = __ffma2_rn(vf[c], pp, o2[g][c]);
+        }
+      }
+    }
+    __syncwarp();
+    if (issued < my_tiles) {
+      vmask[slot] = issue(issued, slot);
+      ++issued;
+    }
+  }
+  if (!ok) {
+    for (int k = consumed + 1; k < issued; ++k) mbar_wait(&bars[k % STAGES], (uint32_t)(k / STAGES) & 1u);
+  }
+
+  // combine within the warp: V partials over the row groups, sums over the lanes of a head
+#pragma unroll
+  for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int c = 0; c < CPL / 2; ++c) {
+        o2[g][c].x += __shfl_xor_sync(0xffffffffu, o2[g][c].x, o);
+        o2[g][c].y += __shfl_xor_sync(0xffffffffu, o2[g][c].y, o);
+      }
+#pragma unroll
+  for (int o = G; o < 32; o <<= 1) l_run += __shfl_xor_sync(0xffffffffu, l_run, o);
+
+  // combine the warps (shared memory reused from the stages)
+  __syncthreads();
+  float* mo = reinterpret_cast<float*>(smem);   // [kWarps][G][D] outputs, then [kWarps][G][2] (m, l)
+  float* mml = mo + kWarps * G * D;
+  if (lane < LPR) {
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int c = 0; c < CPL / 2; ++c)
+        *reinterpret_cast<float2*>(mo + (warp * G + g) * D + lane * CPL + 2 * c) = o2[g][c];
+  }
+  if (lane < G) {
+    mml[(warp * G + lane) * 2 + 0] = m_run;
+    mml[(warp * G + lane) * 2 + 1] = l_run;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < G * D; e += kWarps * 32) {
+    const int g = e / D, c = e - g * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mml[(w * G + g) * 2]);
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float mw = mml[(w * G + g) * 2];
+        if (mw == -INFINITY) continue;
+        const float f = ex2(mw - M);
+        L += mml[(w * G + g) * 2 + 1] * f;
+        O += mo[(w * G + g) * D + c] * f;
+      }
+    }
+    const int hq = h * G + g;
+    const size_t bh = (size_t)b * p.n_q_heads + hq;
+    if (p.splits == 1) {
+      const float r = L > 0.f ? O / L : 0.f;
+      static_cast<KT*>(p.out)[bh * D + c] = E::from_float(r);
+      if (c == 0 && p.lse) p.lse[bh] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+    } else {
+      p.part_o[(bh * p.splits + split) * D + c] = O;
+      if (c == 0) {
+        p.part_ml[(bh * p.splits + split) * 2 + 0] = M;
+        p.part_ml[(bh * p.splits + split) * 2 + 1] = L;
+      }
+    }
+  }
+}
+
+// Log-sum-exp merge of the split partials: one CTA of D threads per query head.
+template <typename KT, int D>
+__global__ void __launch_bounds__(D) attend_merge_kernel(const float* __restrict__ part_o,
+                                                         const float* __restrict__ part_ml, int splits, void* out,
+                                                         float* lse) {
+  using E = Elem<KT>;
+  const size_t bh = blockIdx.x;
+  const int c = threadIdx.x;
+  const float* ml = part_ml + bh * splits * 2;
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[2 * s]);
+  float L = 0.f, O = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < splits; ++s) {
+      const float ms = ml[2 * s];
+      if (ms == -INFINITY) continue;
+      const float f = ex2(ms - M);
+      L += ml[2 * s + 1] * f;
+      O += part_o[(bh * splits + s) * D + c] * f;
+    }
+  }
+  static_cast<KT*>(out)[bh * D + c] = E::from_float(L > 0.f ? O / L : 0.f);
+  if (c == 0 && lse) lse[bh] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+}
+
+template <typename KT, int D, int G>
+cudaError_t launch_t(const AttParams& p, cudaStream_t s) {
+  constexpr int ROW_BYTES = D * Elem<KT>::kBytes;
+  constexpr int TILE_BYTES = 2 * kTile * ROW_BYTES;
+  constexpr int STAGES = 2;
+  auto kern = attend_kernel<KT, D, G, STAGES>;
+  size_t smem = (size_t)kWarps * STAGES * TILE_BYTES + kWarps * STAGES * 8 + (size_t)kWarps * (kTile * G + G) * 4;
+  const size_t merge = (size_t)kWarps * G * (D + 2) * 4;
+  if (smem < merge) smem = merge;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(p.splits, p.batch * p.n_kv), kWarps * 32, smem, s>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.splits == 1) return e;
+  attend_merge_kernel<KT, D><<<p.batch * p.n_q_heads, D, 0, s>>>(p.part_o, p.part_ml, p.splits, p.out, p.lse);
+  return cudaGetLastError();
+}
+
+template <typename KT, int D>
+cudaError_t dispatch_g(int G, const AttParams& p, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_t<KT, D, 1>(p, s);
+    case 2: return launch_t<KT, D, 2>(p, s);
+    case 4: return launch_t<KT, D, 4>(p, s);
+    case 8: return launch_t<KT, D, 8>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail) {
+  AttendPlan pl{1, 64, 0};
+  const long rows = (long)C + (max_tail > 0 ? max_tail : 0);
+  const long units = (long)batch * n_kv_heads;
+  if (rows <= 0 || units <= 0) return pl;
+  const int quantum = kTile * kWarps;   // 64 rows: one tile per warp
+  long per = (rows * units + kTargetCtas - 1) / kTargetCtas;
+  per = ((per + quantum - 1) / quantum) * quantum;
+  if (per < quantum) per = quantum;
+  if (per > rows) per = ((rows + quantum - 1) / quantum) * quantum;
+  pl.rows_per_split = (int)per;
+  pl.splits = (int)((rows + per - 1) / per);
+  if (pl.splits > 1) {
+    const size_t o = (size_t)batch * n_q_heads * pl.splits * head_dim * 4;
+    const size_t ml = (size_t)batch * n_q_heads * pl.splits * 2 * 4;
+    pl.workspace_bytes = ((o + 255) / 256) * 256 + ((ml + 255) / 256) * 256;
+  }
+  return pl;
+}
+
+cudaError_t launch_attend(const void* q, int q_f32, int n_q_heads, const KvView& kv, const int32_t* idx,
+                          const int32_t* count, int C, const int32_t* tail_begin, int max_tail, void* out,
+                          float* lse, void* workspace, const AttendPlan& plan, cudaStream_t s) {
+  AttParams p;
+  p.q = q;
+  p.q_f32 = q_f32;
+  p.n_q_heads = n_q_heads;
+  p.k = static_cast<const uint8_t*>(kv.k);
+  p.v = static_cast<const uint8_t*>(kv.v);
+  p.batch = kv.batch;
+  p.n_kv = kv.n_kv;
+  p.t_max = kv.t_max;
+  p.page_size = kv.page_size;
+  p.max_pages = kv.max_pages;
+  p.n_pages = kv.n_pages;
+  p.page_table = kv.page_table;
+  p.seq_lens = kv.seq_lens;
+  p.idx = idx;
+  p.count = count;
+  p.C = C;
+  p.tail_begin = tail_begin;
+  p.max_tail = tail_begin ? max_tail : 0;
+  p.splits = plan.splits;
+  p.rows_per_split = plan.rows_per_split;
+  if (plan.splits > 1) {
+    const size_t o = (size_t)kv.batch * n_q_heads * plan.splits * kv.head_dim * 4;
+    p.part_o = static_cast<float*>(workspace);
+    p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ((o + 255) / 256) * 256);
+  } else {
+    p.part_o = nullptr;
+    p.part_ml = nullptr;
+  }
+  p.out = out;
+  p.lse = lse;
+  p.qscale = kLog2e / sqrtf((float)kv.head_dim);
+  const int G = n_q_heads / kv.n_kv;
+  if (kv.kv_f32) return kv.head_dim == 64 ? dispatch_g<float, 64>(G, p, s) : dispatch_g<float, 128>(G, p, s);
+  return kv.head_dim == 64 ? dispatch_g<__nv_bfloat16, 64>(G, p, s) : dispatch_g<__nv_bfloat16, 128>(G, p, s);
+}
+
+ASP_STATUS_READER(read_status_attend)
+
+}  // namespace asp

@@ -1,0 +1,89 @@
+// asp_internal.h -- launchers shared between the libasp translation units.
+// Each launcher assumes its arguments were validated by the C ABI layer
+// (asp_api.cu) and returns the CUDA error of its launch.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "asp.h"
+
+namespace asp {
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Per-file device status readers (OR into *bits, then clear).
+cudaError_t read_status_predict(cudaStream_t s, int* bits);
+cudaError_t read_status_score(cudaStream_t s, int* bits);
+cudaError_t read_status_select(cudaStream_t s, int* bits);
+cudaError_t read_status_attend(cudaStream_t s, int* bits);
+cudaError_t read_status_quest(cudaStream_t s, int* bits);
+
+// ---- step 1 -----------------------------------------------------------------
+struct PredictArgs {
+  float* qhist;
+  int ring_start;
+  const void* q_new;      // may be null
+  int q_new_f32;          // 1: fp32, 0: bf16
+  int n_heads;            // batch * n_q_heads
+  int W;
+  int head_dim;
+  int n_win;
+  int windows[8];
+  int wmax;
+  double lam;
+  int coef_raw;
+  float* qpred;
+};
+cudaError_t launch_predict(const PredictArgs& a, cudaStream_t s);
+
+// ---- step 2 -----------------------------------------------------------------
+struct KvView {
+  const void* k;
+  const void* v;
+  int kv_f32;             // 1: fp32, 0: bf16
+  int batch, n_kv, head_dim, t_max;
+  int page_size, max_pages, n_pages;
+  const int32_t* page_table;
+  const int32_t* seq_lens;   // may be null (all t_max)
+};
+cudaError_t launch_score(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s);
+
+// ---- step 3 -----------------------------------------------------------------
+// Selects `c_units` units per row out of ceil(T_b / expand) scores (row stride
+// `row_stride`) and writes each chosen unit u as the tokens u*expand + i (i <
+// expand, tokens >= T_b written as -1), ascending; out row stride c_units*expand.
+struct SelectArgs {
+  const float* scores;
+  int row_stride;
+  const int32_t* seq_lens;  // may be null
+  int t_max;
+  int rows_per_seq;          // n_kv_heads
+  int n_rows;                // batch * n_kv_heads
+  int c_units;
+  int expand;
+  int32_t* idx;
+  int32_t* count;
+};
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
+bool select_supported(int t_max, int expand);
+
+// ---- step 4 -----------------------------------------------------------------
+struct AttendPlan {
+  int splits;
+  int rows_per_split;
+  size_t workspace_bytes;
+};
+AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail);
+cudaError_t launch_attend(const void* q, int q_f32, int n_q_heads, const KvView& kv, const int32_t* idx,
+                          const int32_t* count, int C, const int32_t* tail_begin, int max_tail, void* out,
+                          float* lse, void* workspace, const AttendPlan& plan, cudaStream_t s);
+
+// ---- comparison path ----------------------------------------------------------
+cudaError_t launch_quest_meta(const KvView& kv, int quest_page, void* meta, cudaStream_t s);
+cudaError_t launch_quest_score(const void* q, int q_f32, int n_q_heads, const KvView& kv, const void* meta,
+                               int quest_page, float* page_scores, cudaStream_t s);
+
+}  // namespace asp
