@@ -183,7 +183,8 @@ ASP_API asp_status asp_select_topk(const float* scores, const int32_t* seq_lens,
  * An empty S gives out = 0 and lse = -inf.  Split-K over S with a log-sum-exp merge;
  * fp32 accumulation.
  * q          : device [batch, n_q_heads, head_dim] of q_dtype (bf16 or fp32).
- * idx, count : as written by asp_select_topk (idx row stride C).
+ * idx, count : as written by asp_select_topk (idx row stride C); the first count
+ *              entries of a row must be distinct.  May be NULL when C == 0.
  * tail_begin : device int32 [batch] or NULL (no tail); max_tail bounds T_b - tail_begin
  *              (longer tails are truncated and flagged).  max_tail = t_max with
  *              tail_begin = 0 and count = 0 gives dense attention.

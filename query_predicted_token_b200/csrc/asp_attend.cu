@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(AttParams p) {
   const int b = unit / p.n_kv, h = unit - b * p.n_kv;
   int T = p.seq_lens ? p.seq_lens[b] : p.t_max;
   T = T < 0 ? 0 : (T > p.t_max ? p.t_max : T);
-  int n_sel = p.count[unit];
+  int n_sel = (p.C > 0 && p.count) ? p.count[unit] : 0;
   n_sel = n_sel < 0 ? 0 : (n_sel > p.C ? p.C : n_sel);
   int tb = T;
   if (p.tail_begin) {
@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(AttParams p) {
   const int r0 = split * p.rows_per_split;
   const int r1 = min(n_rows, r0 + p.rows_per_split);
   const int n_tiles = r1 > r0 ? (r1 - r0 + kTile - 1) / kTile : 0;
-  const int32_t* idx_row = p.idx + (size_t)unit * p.C;
+  const int32_t* idx_row = n_sel ? p.idx + (size_t)unit * p.C : nullptr;
 
   if (lane == 0) {
     for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);

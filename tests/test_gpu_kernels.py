@@ -1,0 +1,303 @@
+"""Parity of each CUDA step with the oracle on small seeded inputs (GPU).
+
+Sizes span several 16-row blocks / tiles, ragged tails, empty sequences and
+every supported (dtype, head_dim, group) combination.  All inputs come from
+the seeded generators; all calls go through the C ABI.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import query_predicted_token_b200 as asp
+from parity_util import (OUT_ATOL, assert_lse_close, assert_out_close, assert_pred_close, assert_scores_close,
+                         assert_valid_topk, host_sequences, np64)
+from synth import random_selection, score_rows
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from query_predicted_token_b200 import build
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    asp.lib()
+    yield
+    assert asp.device_status() == 0
+
+
+def _gen(seed):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return g
+
+
+def make_cache(B, Hkv, d, T, dtype, lens, page_size=0, seed=0):
+    """Small KV cache on the GPU (contiguous or paged with a shuffled table)."""
+    g = _gen(seed)
+    if page_size == 0:
+        k = torch.randn(B, Hkv, T, d, generator=g).to(dtype)
+        v = torch.randn(B, Hkv, T, d, generator=g).to(dtype)
+        kvd = dict(k=k.to(DEV), v=v.to(DEV), seq_lens=torch.tensor(lens, dtype=torch.int32, device=DEV),
+                   page_table=None, page_size=0)
+        return kvd, asp.KV(kvd["k"], kvd["v"], kvd["seq_lens"])
+    P = page_size
+    maxp = (T + P - 1) // P
+    per = [(t + P - 1) // P for t in lens]
+    n = max(1, sum(per))
+    perm = torch.randperm(n, generator=g).to(torch.int32)
+    table = torch.full((B, maxp), -1, dtype=torch.int32)
+    off = 0
+    for b, c in enumerate(per):
+        table[b, :c] = perm[off:off + c]
+        off += c
+    k = torch.randn(n, Hkv, P, d, generator=g).to(dtype)
+    v = torch.randn(n, Hkv, P, d, generator=g).to(dtype)
+    kvd = dict(k=k.to(DEV), v=v.to(DEV), seq_lens=torch.tensor(lens, dtype=torch.int32, device=DEV),
+               page_table=table.to(DEV), page_size=P)
+    return kvd, asp.KV(kvd["k"], kvd["v"], kvd["seq_lens"], kvd["page_table"], t_max=T)
+
+
+CASES = [(dt, d, G) for dt in (torch.bfloat16, torch.float32) for d in (64, 128) for G in (1, 2, 4, 8)]
+
+
+@pytest.mark.parametrize("dtype,d,G", CASES)
+@pytest.mark.parametrize("page_size", [0, 16, 32])
+def test_score_keys(dtype, d, G, page_size):
+    B, Hkv, T = 3, 2, 1000
+    lens = [1000, 517, 1] if page_size == 0 else [1000, 530, 17]
+    kvd, kv = make_cache(B, Hkv, d, T, dtype, lens, page_size, seed=G * 10 + d)
+    qpred = torch.randn(B, Hkv * G, d, generator=_gen(5)).to(DEV)
+    scores = torch.full((B, Hkv, T), float("nan"), device=DEV)
+    asp.score_keys(qpred, kv, scores)
+    torch.cuda.synchronize()
+    keys, _ = host_sequences(kvd)
+    ref = oracle.score_keys(np64(qpred), [keys[b] for b in range(B)], T)
+    got = scores.cpu().numpy()
+    for b in range(B):
+        for h in range(Hkv):
+            Tb = lens[b]
+            assert_scores_close(got[b, h, :Tb], ref[b, h, :Tb], np64(qpred[b, h * G:(h + 1) * G]), keys[b][h],
+                                what=f"b{b} h{h}")
+            assert np.isnan(got[b, h, Tb:]).all()      # entries past T_b are not written
+
+
+def test_score_empty_sequence_writes_nothing():
+    kvd, kv = make_cache(2, 2, 128, 64, torch.bfloat16, [0, 40])
+    qpred = torch.randn(2, 8, 128, generator=_gen(1)).to(DEV)
+    scores = torch.full((2, 2, 64), float("nan"), device=DEV)
+    asp.score_keys(qpred, kv, scores)
+    torch.cuda.synchronize()
+    assert torch.isnan(scores[0]).all() and not torch.isnan(scores[1, :, :40]).any()
+
+
+@pytest.mark.parametrize("T,C", [(1, 1), (100, 7), (2048, 2048), (5000, 2048), (5000, 4999), (32768, 2048),
+                                 (65536, 2048), (100003, 1000), (70000, 65536)])
+@pytest.mark.parametrize("kind", ["normal", "ties", "special", "equal"])
+def test_select_topk_bit_exact(T, C, kind):
+    rows = 4
+    s = score_rows(rows, T, seed=T + C, kind=kind)
+    lens = torch.tensor([T, max(1, T // 3), max(1, T - 5), min(T, C)], dtype=torch.int32)
+    sc = s.to(DEV).view(rows, 1, T).repeat(1, 2, 1).contiguous()        # 2 KV heads, same row
+    idx = torch.full((rows, 2, C), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.full((rows, 2), -7, dtype=torch.int32, device=DEV)
+    asp.select_topk(sc, lens.to(DEV), C, idx, cnt)
+    torch.cuda.synchronize()
+    ref_idx, ref_cnt = oracle.select_topk(np.repeat(s.numpy()[:, None, :], 2, axis=1), lens.tolist(), C)
+    assert np.array_equal(cnt.cpu().numpy(), ref_cnt)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+
+
+def test_select_without_seq_lens_uses_t_max():
+    s = score_rows(3, 3000, seed=1).to(DEV).view(3, 1, 3000)
+    idx = torch.empty(3, 1, 100, dtype=torch.int32, device=DEV)
+    cnt = torch.empty(3, 1, dtype=torch.int32, device=DEV)
+    asp.select_topk(s, None, 100, idx, cnt)
+    ref_idx, ref_cnt = oracle.select_topk(s.cpu().numpy(), [3000] * 3, 100)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx) and np.array_equal(cnt.cpu().numpy(), ref_cnt)
+
+
+def test_select_empty_rows():
+    s = score_rows(2, 50, seed=3).to(DEV).view(2, 1, 50)
+    idx = torch.full((2, 1, 8), 5, dtype=torch.int32, device=DEV)
+    cnt = torch.full((2, 1), 5, dtype=torch.int32, device=DEV)
+    asp.select_topk(s, torch.tensor([0, 3], dtype=torch.int32, device=DEV), 8, idx, cnt)
+    assert cnt.cpu().tolist() == [[0], [3]]
+    assert idx[0].cpu().tolist() == [[-1] * 8] and idx[1].cpu().tolist() == [[0, 1, 2] + [-1] * 5]
+
+
+@pytest.mark.parametrize("dtype,d,G", CASES)
+@pytest.mark.parametrize("page_size", [0, 16])
+@pytest.mark.parametrize("C", [1, 37, 300])
+def test_sparse_attend(dtype, d, G, page_size, C):
+    B, Hkv, T = 3, 2, 700
+    lens = [700, 333, 5]
+    kvd, kv = make_cache(B, Hkv, d, T, dtype, lens, page_size, seed=C + d)
+    q = torch.randn(B, Hkv * G, d, generator=_gen(C)).to(dtype).to(DEV)
+    idx, cnt = random_selection(B, Hkv, C, lens, seed=C * 7 + G)
+    out = torch.empty(B, Hkv * G, d, dtype=dtype, device=DEV)
+    lse = torch.empty(B, Hkv * G, device=DEV)
+    ws = torch.empty(max(16, asp.attend_workspace_bytes(B, Hkv * G, Hkv, d, C)), dtype=torch.uint8, device=DEV)
+    asp.sparse_attend(q, kv, idx.to(DEV), cnt.to(DEV), C, out, lse, workspace=ws)
+    torch.cuda.synchronize()
+    keys, vals = host_sequences(kvd)
+    ref, ref_lse = oracle.sparse_attend(np64(q), [keys[b] for b in range(B)], [vals[b] for b in range(B)],
+                                        idx.numpy(), cnt.numpy())
+    assert_out_close(out, ref, dtype, f"{dtype} d{d} G{G} P{page_size} C{C}")
+    assert_lse_close(lse, ref_lse)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_sparse_attend_many_splits_and_tail(dtype):
+    B, Hkv, G, d, T = 2, 2, 4, 128, 6000
+    lens = [6000, 4100]
+    kvd, kv = make_cache(B, Hkv, d, T, dtype, lens, 16, seed=11)
+    C, max_tail = 2048, 64
+    # the selection was made on a snapshot; tokens from tail_begin on are attended in full
+    tail_begin = torch.tensor([5990, 4100 - 64], dtype=torch.int32)
+    idx, cnt = random_selection(B, Hkv, C, tail_begin.tolist(), seed=3)
+    q = torch.randn(B, Hkv * G, d, generator=_gen(9)).to(dtype).to(DEV)
+    out = torch.empty(B, Hkv * G, d, dtype=dtype, device=DEV)
+    lse = torch.empty(B, Hkv * G, device=DEV)
+    ws = torch.empty(asp.attend_workspace_bytes(B, Hkv * G, Hkv, d, C, max_tail), dtype=torch.uint8, device=DEV)
+    asp.sparse_attend(q, kv, idx.to(DEV), cnt.to(DEV), C, out, lse, tail_begin.to(DEV), max_tail, ws)
+    torch.cuda.synchronize()
+    keys, vals = host_sequences(kvd)
+    ref, ref_lse = oracle.sparse_attend(np64(q), [keys[0], keys[1]], [vals[0], vals[1]], idx.numpy(), cnt.numpy(),
+                                        tail_begin.tolist())
+    assert_out_close(out, ref, dtype)
+    assert_lse_close(lse, ref_lse)
+
+
+def test_dense_attention_through_the_tail():
+    """count = 0 and tail_begin = 0 attends every token: full attention."""
+    B, Hkv, G, d, T = 2, 2, 2, 64, 3000
+    kvd, kv = make_cache(B, Hkv, d, T, torch.float32, [3000, 1234], seed=4)
+    q = torch.randn(B, Hkv * G, d, generator=_gen(2)).to(DEV)
+    zero = torch.zeros(B, dtype=torch.int32, device=DEV)
+    out = torch.empty(B, Hkv * G, d, device=DEV)
+    ws = torch.empty(max(16, asp.attend_workspace_bytes(B, Hkv * G, Hkv, d, 0, T)), dtype=torch.uint8, device=DEV)
+    asp.sparse_attend(q, kv, None, None, 0, out, None, zero, T, ws)
+    torch.cuda.synchronize()
+    keys, vals = host_sequences(kvd)
+    Kt = [torch.from_numpy(keys[b]) for b in range(B)]
+    Vt = [torch.from_numpy(vals[b]) for b in range(B)]
+    for b in range(B):
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(np64(q[b]))[:, None, :], Kt[b].repeat_interleave(G, 0), Vt[b].repeat_interleave(G, 0))
+        assert (np64(out[b]) - ref[:, 0].numpy()).__abs__().max() <= OUT_ATOL[torch.float32]
+
+
+def test_attend_flags_out_of_range_indices_and_skips_them():
+    B, Hkv, G, d, T = 1, 1, 2, 128, 200
+    kvd, kv = make_cache(B, Hkv, d, T, torch.bfloat16, [200], seed=8)
+    idx = torch.tensor([[[3, 10, 250, 60, -4]]], dtype=torch.int32)
+    cnt = torch.tensor([[5]], dtype=torch.int32)
+    q = torch.randn(B, Hkv * G, d, generator=_gen(3)).to(torch.bfloat16).to(DEV)
+    out = torch.empty(B, Hkv * G, d, dtype=torch.bfloat16, device=DEV)
+    assert asp.device_status() == 0
+    asp.sparse_attend(q, kv, idx.to(DEV), cnt.to(DEV), 5, out)
+    bits = asp.device_status()
+    assert bits & asp.ASP_DEV_BAD_INDEX
+    keys, vals = host_sequences(kvd)
+    ref, _ = oracle.sparse_attend(np64(q), [keys[0]], [vals[0]], np.array([[[3, 10, 60]]]), np.array([[3]]))
+    assert_out_close(out, ref, torch.bfloat16)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("W,windows", [(1, (1,)), (8, (4, 8)), (16, (4, 8, 16)), (16, (2, 5, 11)), (32, (1, 7, 32))])
+@pytest.mark.parametrize("coef", ["softmax", "raw"])
+def test_predict_query(d, W, windows, coef):
+    B, Hq = 2, 6
+    g = _gen(W * 100 + d)
+    q = [torch.randn(B, Hq, d, generator=g)]
+    for _ in range(W):
+        q.append(0.9 * q[-1] + 0.1 * torch.randn(B, Hq, d, generator=g))
+    hist = torch.stack(q, dim=2)                          # [B, Hq, W+1, d] oldest first
+    for ring in (0, W // 2 + (W > 0), W):
+        ring = ring % (W + 1)
+        slots = torch.roll(hist, shifts=ring, dims=2)      # slot (ring + s) % (W+1) holds s-th oldest
+        qhist = slots.contiguous().to(DEV)
+        qpred = torch.empty(B, Hq, d, device=DEV)
+        cfg = asp.PredCfg(W, windows, 1e-2, coef)
+        asp.predict_query(qhist, ring, cfg, qpred)
+        torch.cuda.synchronize()
+        ref = oracle.predict_query(hist.double().numpy(), windows, 1e-2, coef)
+        assert_pred_close(qpred.cpu().numpy(), ref, f"W{W} {windows} ring{ring} {coef}")
+        assert torch.equal(qhist.cpu(), slots)             # read-only without q_new
+
+
+@pytest.mark.parametrize("qdtype", [torch.float32, torch.bfloat16])
+def test_predict_query_pushes_the_new_query(qdtype):
+    B, Hq, d, W, windows = 2, 4, 128, 16, (4, 8, 16)
+    g = _gen(77)
+    seq = [torch.randn(B, Hq, d, generator=g)]
+    for _ in range(W + 1):
+        seq.append(0.9 * seq[-1] + 0.1 * torch.randn(B, Hq, d, generator=g))
+    hist0 = torch.stack(seq[:W + 1], dim=2)
+    q_new = seq[W + 1].to(qdtype)
+    ring = 5
+    qhist = torch.roll(hist0, shifts=ring, dims=2).contiguous().to(DEV)
+    qpred = torch.empty(B, Hq, d, device=DEV)
+    asp.predict_query(qhist, ring, asp.PredCfg(W, windows, 1e-2), qpred, q_new=q_new.to(DEV))
+    torch.cuda.synchronize()
+    hist1 = torch.cat([hist0[:, :, 1:], q_new.float()[:, :, None]], dim=2)
+    ref = oracle.predict_query(hist1.double().numpy(), windows, 1e-2)
+    assert_pred_close(qpred.cpu().numpy(), ref)
+    assert torch.equal(qhist.cpu()[:, :, ring], q_new.float())          # oldest slot overwritten
+    assert torch.equal(torch.roll(qhist.cpu(), shifts=-(ring + 1), dims=2), hist1)
+
+
+@pytest.mark.parametrize("dtype,d,G", [(torch.bfloat16, 128, 4), (torch.bfloat16, 128, 8), (torch.float32, 64, 2)])
+@pytest.mark.parametrize("page_size", [0, 16])
+def test_quest_path(dtype, d, G, page_size):
+    B, Hkv, T, P, C = 2, 2, 1500, 16, 256
+    lens = [1500, 777]
+    kvd, kv = make_cache(B, Hkv, d, T, dtype, lens, page_size, seed=31)
+    npm = (T + P - 1) // P
+    meta = torch.zeros(B, Hkv, npm, 2, d, dtype=dtype, device=DEV)
+    asp.quest_build_meta(kv, P, meta)
+    q = torch.randn(B, Hkv * G, d, generator=_gen(4)).to(dtype).to(DEV)
+    ps = torch.full((B, Hkv, npm), float("nan"), device=DEV)
+    cap = ((C + P - 1) // P) * P
+    idx = torch.empty(B, Hkv, cap, dtype=torch.int32, device=DEV)
+    cnt = torch.empty(B, Hkv, dtype=torch.int32, device=DEV)
+    asp.quest_select(q, kv, meta, P, C, ps, idx, cnt)
+    torch.cuda.synchronize()
+    keys, _ = host_sequences(kvd)
+    for b in range(B):
+        for h in range(Hkv):
+            kmin, kmax = oracle.quest_meta(keys[b][h], P)
+            n = kmin.shape[0]
+            assert np.array_equal(np64(meta[b, h, :n, 0]), kmin) and np.array_equal(np64(meta[b, h, :n, 1]), kmax)
+            qg = np64(q[b, h * G:(h + 1) * G])
+            ref_ps = oracle.quest_page_scores(qg, kmin, kmax)
+            got_ps = ps[b, h, :n].cpu().numpy()
+            # the bound is a sum of |q| |k| terms: same tolerance rule as the key scores, on page rows
+            rows = np.concatenate([kmin, kmax], axis=1)
+            assert_scores_close(got_ps, ref_ps, np.concatenate([qg, qg], axis=1), rows / math.sqrt(2), f"pages b{b}h{h}")
+            m = cnt[b, h].item()
+            chosen = idx[b, h, :m].cpu().numpy()
+            pages = np.unique(chosen // P)
+            # the kept pages are the best ceil(C/P) of the GPU's own page scores, lowest index on ties
+            page_idx = np.full(npm, -1, dtype=np.int64)
+            page_idx[:pages.size] = pages
+            assert_valid_topk(got_ps, n, (C + P - 1) // P, page_idx[:(C + P - 1) // P], pages.size, f"b{b}h{h}")
+            expect = (pages[:, None] * P + np.arange(P)[None, :]).reshape(-1)
+            expect = expect[expect < lens[b]]
+            assert chosen.tolist() == expect.tolist() and m == expect.size
+            assert (idx[b, h, m:] == -1).all()
+
+
+def test_wait_selection_times_out_then_completes():
+    s = torch.cuda.Stream()
+    ev = asp.make_event()
+    with torch.cuda.stream(s):
+        torch.cuda._sleep(200_000_000)           # ~0.1 s of GPU spinning, bounded
+        ev.record(s)
+    assert asp.wait_selection(ev, 10) == asp._lib.ASP_ERR_TIMEOUT
+    assert asp.wait_selection(ev, 30_000_000) == asp._lib.ASP_OK

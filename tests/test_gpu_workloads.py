@@ -1,0 +1,167 @@
+"""The decode path at the workloads' full sizes, in the bench's launch configuration (GPU).
+
+One ``asp_decode_step`` per test: attention of step t over a seeded selection
+on the main stream, prediction / scoring / selection for step t+1 on the side
+stream.  The oracle recomputes sampled outputs one (sequence, KV head) unit at
+a time; the whole selection is checked as a property of the GPU's own scores
+and against the oracle's selection where the oracle's scores leave no near-tie.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import query_predicted_token_b200 as asp
+import synth
+from parity_util import (assert_lse_close, assert_out_close, assert_pred_close, assert_scores_close,
+                         assert_valid_topk, host_sequences, np64)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from query_predicted_token_b200 import build
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    yield
+    assert asp.device_status() == 0
+
+
+def run_step(wl, kvd, tail=0, sample_units=((0, 0),), steps=1):
+    """One decode step of a workload; checks it against the oracle on sampled units."""
+    B, Hq, Hkv, d = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+    G = Hq // Hkv
+    lens = kvd["seq_lens"].cpu()
+    kv = asp.KV(kvd["k"], kvd["v"], kvd["seq_lens"], kvd["page_table"], t_max=wl.t_max)
+    qhist, q_next = synth.query_history(wl, steps=1)
+    q_t = q_next[0].to(wl.torch_dtype())
+    tail_begin = (lens - tail).clamp(min=0) if tail else None
+    snap = tail_begin.tolist() if tail else lens.tolist()
+    idx0, cnt0 = synth.random_selection(B, Hkv, wl.C, snap, seed=wl.seed + 99)
+    st = asp.DecodeState(kv, Hq, asp.PredCfg(wl.W, wl.windows, wl.lam), wl.C, qhist.to(DEV).contiguous(),
+                         max_tail=tail, tail_begin=tail_begin.to(torch.int32).to(DEV) if tail else None)
+    st.set_selection(idx0.to(DEV), cnt0.to(DEV))
+    out = torch.empty(B, Hq, d, dtype=wl.torch_dtype(), device=DEV)
+    lse = torch.empty(B, Hq, device=DEV)
+    st.step(q_t.to(DEV), out, lse)
+    assert asp.wait_selection(st.ev_sel_done, 60_000_000) == 0
+    torch.cuda.synchronize()
+    assert asp.device_status() == 0
+
+    # step 1: predicted query of every head
+    hist1 = torch.cat([qhist[:, :, 1:], q_t.float()[:, :, None]], dim=2)
+    ref_pred = oracle.predict_query(hist1.double().numpy(), wl.windows, wl.lam)
+    assert_pred_close(st.qpred.cpu().numpy(), ref_pred, wl.name)
+
+    scores = st.scores.cpu().numpy()
+    idx1, cnt1 = (t.cpu().numpy() for t in st.selection)
+    # step 3 on every row: the chosen set is the top C of the GPU's own scores
+    for b in range(B):
+        for h in range(Hkv):
+            assert_valid_topk(scores[b, h], int(lens[b]), wl.C, idx1[b, h], int(cnt1[b, h]), f"{wl.name} b{b}h{h}")
+
+    bs = sorted({b for b, _ in sample_units})
+    keys, vals = host_sequences(kvd, bs)
+    qn = np64(q_t)
+    gpu_pred = st.qpred.cpu().double().numpy()
+    for b, h in sample_units:
+        Tb = int(lens[b])
+        K, V = keys[b][h], vals[b][h]
+        qg = gpu_pred[b, h * G:(h + 1) * G]
+        # step 2: scores of this unit for every token (same predicted query on both sides)
+        ref_s = oracle.score_row(qg, K)
+        assert_scores_close(scores[b, h, :Tb], ref_s, qg, K, f"{wl.name} b{b}h{h}")
+        # step 3 against the oracle's own selection from its float64 scores: identical
+        # except where the oracle's scores are closer than the score tolerance
+        ref_sel, _ = oracle.select_row(ref_s.astype(np.float32), Tb, wl.C)
+        got_sel = idx1[b, h, :int(cnt1[b, h])]
+        diff = np.setxor1d(ref_sel, got_sel)
+        if diff.size:
+            thr = np.sort(ref_s)[::-1][min(wl.C, Tb) - 1]
+            assert np.all(np.abs(ref_s[diff] - thr) <= 1e-3 * abs(thr) + 1e-5), f"{wl.name}: selection differs"
+        # step 4: attention of step t over the seeded selection (+ tail)
+        S = oracle.attend.attended_set(idx0[b, h].numpy(), int(cnt0[b, h]), snap[b] if tail else None, Tb)
+        ref_o, ref_l = oracle.attend_set(qn[b, h * G:(h + 1) * G], K, V, S)
+        assert_out_close(out[b, h * G:(h + 1) * G], ref_o, wl.torch_dtype(), f"{wl.name} out b{b}h{h}")
+        assert_lse_close(lse[b, h * G:(h + 1) * G], ref_l)
+    return st
+
+
+def test_tiny_f32_t512_two_steps_against_the_oracle_pipeline():
+    wl = synth.workload("tiny_f32_t512")
+    kvd = synth.kv_cache(wl, DEV)
+    units = [(0, 0), (0, 1)]
+    st = run_step(wl, kvd, sample_units=units)
+    # the whole two-step schedule against the oracle's own pipeline
+    qhist, q_next = synth.query_history(wl, steps=2)
+    keys, vals = host_sequences(kvd)
+    idx0, cnt0 = synth.random_selection(1, 2, wl.C, [wl.t_max], seed=wl.seed + 99)
+    r1 = oracle.decode_step(q_next[0].numpy(), qhist.numpy(), [keys[0]], [vals[0]], idx0.numpy(), cnt0.numpy(),
+                            wl.C, wl.windows, wl.lam, wl.t_max)
+    idx1, cnt1 = (t.cpu().numpy() for t in st.selection)
+    assert np.array_equal(idx1, r1["idx"]) and np.array_equal(cnt1, r1["count"])
+    out2 = torch.empty(1, 4, 64, device=DEV)
+    st.step(q_next[1].to(DEV), out2)
+    torch.cuda.synchronize()
+    r2 = oracle.decode_step(q_next[1].numpy(), r1["qhist"], [keys[0]], [vals[0]], r1["idx"], r1["count"], wl.C,
+                            wl.windows, wl.lam, wl.t_max)
+    assert_out_close(out2, r2["out"], torch.float32, "step 2")
+    idx2, cnt2 = (t.cpu().numpy() for t in st.selection)
+    assert np.array_equal(idx2, r2["idx"]) and np.array_equal(cnt2, r2["count"])
+
+
+def test_qwen3_8b_shaped_32k():
+    wl = synth.workload("qwen3_8b_shaped_32k")
+    kvd = synth.kv_cache(wl, DEV)
+    run_step(wl, kvd, sample_units=[(0, 0), (5, 7), (7, 3)])
+
+
+def test_qwen3_32b_shaped_32k():
+    wl = synth.workload("qwen3_32b_shaped_32k")
+    kvd = synth.kv_cache(wl, DEV)
+    run_step(wl, kvd, sample_units=[(0, 0), (15, 7)])
+
+
+def test_longcot_ragged_paged_b64():
+    wl = synth.workload("longcot_ragged_paged_b64")
+    kvd = synth.kv_cache(wl, DEV)
+    lens = kvd["seq_lens"].cpu()
+    b_long, b_short = int(lens.argmax()), int(lens.argmin())
+    run_step(wl, kvd, tail=1, sample_units=[(b_long, 0), (b_short, 5)])
+    del kvd
+    torch.cuda.empty_cache()
+
+
+def test_quest_page_scan_8b_32k():
+    wl = synth.workload("quest_page_scan_8b_32k")
+    kvd = synth.kv_cache(wl, DEV, layout="contiguous")
+    B, Hq, Hkv, d, P = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, 16
+    G = Hq // Hkv
+    kv = asp.KV(kvd["k"], kvd["v"], kvd["seq_lens"])
+    npm = wl.t_max // P
+    meta = torch.empty(B, Hkv, npm, 2, d, dtype=torch.bfloat16, device=DEV)
+    asp.quest_build_meta(kv, P, meta)
+    _, q_next = synth.query_history(wl, steps=1)
+    q = q_next[0].to(torch.bfloat16).to(DEV)
+    ps = torch.empty(B, Hkv, npm, device=DEV)
+    idx = torch.empty(B, Hkv, wl.C, dtype=torch.int32, device=DEV)
+    cnt = torch.empty(B, Hkv, dtype=torch.int32, device=DEV)
+    asp.quest_select(q, kv, meta, P, wl.C, ps, idx, cnt)
+    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=DEV)
+    ws = torch.empty(asp.attend_workspace_bytes(B, Hq, Hkv, d, wl.C), dtype=torch.uint8, device=DEV)
+    asp.sparse_attend(q, kv, idx, cnt, wl.C, out, workspace=ws)
+    torch.cuda.synchronize()
+    assert (cnt == wl.C).all()
+    keys, vals = host_sequences(kvd, [2])
+    for h in (0, 6):
+        kmin, kmax = oracle.quest_meta(keys[2][h], P)
+        assert np.array_equal(np64(meta[2, h, :, 0]), kmin) and np.array_equal(np64(meta[2, h, :, 1]), kmax)
+        qg = np64(q[2, h * G:(h + 1) * G])
+        sel = idx[2, h].cpu().numpy()
+        pages = np.unique(sel // P)
+        assert pages.size == wl.C // P
+        assert_valid_topk(ps[2, h].cpu().numpy(), npm, wl.C // P, pages, pages.size, "pages")
+        ref_o, _ = oracle.attend_set(qg, keys[2][h], vals[2][h], sel)
+        assert_out_close(out[2, h * G:(h + 1) * G], ref_o, torch.bfloat16, "quest attention")
