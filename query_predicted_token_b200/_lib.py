@@ -256,31 +256,26 @@ class DecodeState:
         self.timing_events = [make_event(True) for _ in range(8)] if timing else None
         self._timing_arr = (c_void_p * 8)(*[event_handle(e) for e in self.timing_events]) if timing else None
 
-    def set_selection(self, idx: torch.Tensor, count: torch.Tensor) -> None:
-        self.idx[self.cur].copy_(idx)
-        self.count[self.cur].copy_(count)
+        self._args = [self._build_args(0), self._build_args(1)]
+        self._fn = lib().asp_decode_step
 
-    def step(self, q_t: torch.Tensor, out: torch.Tensor, lse: Optional[torch.Tensor] = None) -> None:
-        nxt = 1 - self.cur
+    def _build_args(self, cur: int) -> AspDecodeArgs:
+        """The call's arguments for one parity of the double-buffered selection."""
+        nxt = 1 - cur
         a = AspDecodeArgs()
-        a.q_t = _ptr(q_t)
-        a.q_dtype = dtype_code(q_t)
         a.n_q_heads = self.n_q_heads
         a.qhist = _ptr(self.qhist)
-        a.ring_start = self.ring_start
         a.pred = ctypes.pointer(self.cfg.struct)
         a.kv = ctypes.pointer(self.kv.struct)
         a.C = self.C
-        a.idx_cur = _ptr(self.idx[self.cur])
-        a.count_cur = _ptr(self.count[self.cur])
+        a.idx_cur = _ptr(self.idx[cur])
+        a.count_cur = _ptr(self.count[cur])
         a.tail_begin = _ptr(self.tail_begin)
         a.max_tail = self.max_tail
         a.qpred = _ptr(self.qpred)
         a.scores = _ptr(self.scores)
         a.idx_next = _ptr(self.idx[nxt])
         a.count_next = _ptr(self.count[nxt])
-        a.out = _ptr(out)
-        a.lse = _ptr(lse)
         a.workspace = _ptr(self.workspace)
         a.workspace_bytes = self.workspace.numel()
         a.s_main = _stream(self.s_main)
@@ -288,8 +283,21 @@ class DecodeState:
         a.ev_fork = event_handle(self.ev_fork)
         a.ev_sel_done = event_handle(self.ev_sel_done)
         a.timing = ctypes.cast(self._timing_arr, POINTER(c_void_p)) if self._timing_arr is not None else None
-        _check("asp_decode_step", lib().asp_decode_step(ctypes.byref(a)))
-        self.cur = nxt
+        return a
+
+    def set_selection(self, idx: torch.Tensor, count: torch.Tensor) -> None:
+        self.idx[self.cur].copy_(idx)
+        self.count[self.cur].copy_(count)
+
+    def step(self, q_t: torch.Tensor, out: torch.Tensor, lse: Optional[torch.Tensor] = None) -> None:
+        a = self._args[self.cur]
+        a.q_t = q_t.data_ptr()
+        a.q_dtype = dtype_code(q_t)
+        a.out = out.data_ptr()
+        a.lse = lse.data_ptr() if lse is not None else None
+        a.ring_start = self.ring_start
+        _check("asp_decode_step", self._fn(ctypes.byref(a)))
+        self.cur = 1 - self.cur
         self.ring_start = (self.ring_start + 1) % (self.cfg.W + 1)
 
     @property

@@ -3,7 +3,10 @@
 // allocates memory; every error is reported as an asp_status.
 #include <chrono>
 #include <cmath>
+#include <map>
+#include <mutex>
 #include <thread>
+#include <tuple>
 
 #include "asp_common.cuh"
 #include "asp_internal.h"
@@ -19,6 +22,35 @@ int sm_count() {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) cache[dev] = n;
   }
   return cache[dev] > 0 ? cache[dev] : 148;
+}
+
+int prepare_kernel(const void* kern, size_t smem, int threads) {
+  // The dynamic shared-memory limit is one attribute per kernel: keep it at the
+  // largest size requested so far, so that every cached configuration stays valid.
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, size_t> limit;
+  static std::map<std::tuple<const void*, int, size_t, int>, int> occupancy;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  size_t& cur = limit[std::make_pair(kern, dev)];
+  if (smem > cur) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return 0;
+    }
+    cur = smem;
+  }
+  const auto key = std::make_tuple(kern, dev, smem, threads);
+  auto it = occupancy.find(key);
+  if (it != occupancy.end()) return it->second;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  occupancy[key] = per_sm;
+  return per_sm;
 }
 
 }  // namespace asp

@@ -25,7 +25,6 @@ namespace {
 
 constexpr int kTile = 16;
 constexpr int kWarps = 4;
-constexpr int kTargetCtas = 592;   // 4 CTAs per SM of a 148-SM B200
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -412,10 +411,9 @@ cudaError_t launch_t(const AttParams& p, cudaStream_t s) {
   size_t smem = (size_t)kWarps * STAGES * TILE_BYTES + kWarps * STAGES * 8 + (size_t)kWarps * (kTile * G + G) * 4;
   const size_t merge = (size_t)kWarps * G * (D + 2) * 4;
   if (smem < merge) smem = merge;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
   kern<<<dim3(p.splits, p.batch * p.n_kv), kWarps * 32, smem, s>>>(p);
-  e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || p.splits == 1) return e;
   attend_merge_kernel<KT, D><<<p.batch * p.n_q_heads, D, 0, s>>>(p.part_o, p.part_ml, p.splits, p.out, p.lse);
   return cudaGetLastError();
@@ -434,16 +432,22 @@ cudaError_t dispatch_g(int G, const AttParams& p, cudaStream_t s) {
 
 }  // namespace
 
+// Split plan: as many splits per KV head as fit in one wave of resident CTAs on
+// a 148-SM B200 (3 CTAs per SM for G <= 4, 2 for G = 8, set by the registers),
+// each split a multiple of 64 rows (one 16-row tile per warp).  A pure function
+// of the sizes, so the workspace size is known without a device.
 AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail) {
   AttendPlan pl{1, 64, 0};
   const long rows = (long)C + (max_tail > 0 ? max_tail : 0);
   const long units = (long)batch * n_kv_heads;
-  if (rows <= 0 || units <= 0) return pl;
-  const int quantum = kTile * kWarps;   // 64 rows: one tile per warp
-  long per = (rows * units + kTargetCtas - 1) / kTargetCtas;
+  if (rows <= 0 || units <= 0 || n_kv_heads <= 0) return pl;
+  const int G = n_q_heads / n_kv_heads;
+  const long target = 148L * (G >= 8 ? 2 : 3);
+  const int quantum = kTile * kWarps;
+  long splits = target / units;
+  if (splits < 1) splits = 1;
+  long per = (rows + splits - 1) / splits;
   per = ((per + quantum - 1) / quantum) * quantum;
-  if (per < quantum) per = quantum;
-  if (per > rows) per = ((rows + quantum - 1) / quantum) * quantum;
   pl.rows_per_split = (int)per;
   pl.splits = (int)((rows + per - 1) / per);
   if (pl.splits > 1) {

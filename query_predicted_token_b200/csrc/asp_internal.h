@@ -14,6 +14,11 @@ namespace asp {
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
+// One-time launch setup per (kernel, device, dynamic shared memory): raises the
+// kernel's dynamic shared-memory limit and returns its resident CTAs per SM
+// (0 if the configuration cannot launch).  Cached, so launches stay cheap.
+int prepare_kernel(const void* kern, size_t smem, int threads);
+
 // Per-file device status readers (OR into *bits, then clear).
 cudaError_t read_status_predict(cudaStream_t s, int* bits);
 cudaError_t read_status_score(cudaStream_t s, int* bits);

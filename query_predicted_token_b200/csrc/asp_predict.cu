@@ -23,7 +23,8 @@ namespace asp {
 namespace {
 
 constexpr int kWarps = 4;
-constexpr size_t kSolveBytes = 32 * 32 * 8 + 3 * 32 * 8;   // A[32][32], rhs, z, coef (fp64)
+constexpr int kLda = 33;   // row stride (doubles) of the lag Gram: column accesses hit distinct banks
+constexpr size_t kSolveBytes = (32 * kLda + 3 * 32) * 8;   // A[32][33], rhs, 1/diag, spare (fp64)
 
 template <int N, int OFF>
 struct ReduceScatterD {
@@ -62,9 +63,8 @@ __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
   uint8_t* base = smem + warp * (hv_bytes + kSolveBytes);
   float* hv = reinterpret_cast<float*>(base);
   double* A = reinterpret_cast<double*>(base + hv_bytes);
-  double* rhs = A + 32 * 32;
-  double* y = rhs + 32;
-  double* coef = y + 32;
+  double* rhs = A + 32 * kLda;
+  double* invd = rhs + 32;
 
   float* hist = a.qhist + (size_t)head * nslot * D;
   // chronological position s (0 = oldest, W = newest) -> ring slot
@@ -129,34 +129,38 @@ __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
       }
     }
     if (p0 + lane < n_pairs) {
-      if (ti < wm) A[ti * 32 + tj] = vals[0] + (ti == tj ? a.lam : 0.0);
+      if (ti < wm) A[ti * kLda + tj] = vals[0] + (ti == tj ? a.lam : 0.0);
       else rhs[tj] = vals[0];
     }
   }
   __syncwarp();
 
-  // Cholesky A = L L^T in place (lower triangle), right-looking, lane i owns row i.
+  // Cholesky A = L L^T in place (lower triangle), right-looking.  Every lane
+  // computes the pivot; lane i owns row i; column k is broadcast by shuffles.
   for (int k = 0; k < wm; ++k) {
-    if (lane == 0) A[k * 32 + k] = sqrt(A[k * 32 + k]);
-    __syncwarp();
-    const double dkk = A[k * 32 + k];
-    const int i = lane;
-    if (i > k && i < wm) A[i * 32 + k] /= dkk;
-    __syncwarp();
-    if (i > k && i < wm) {
-      const double lik = A[i * 32 + k];
-      for (int j = k + 1; j <= i; ++j) A[i * 32 + j] -= lik * A[j * 32 + k];
+    const double dkk = sqrt(A[k * kLda + k]);
+    const double inv = 1.0 / dkk;
+    double lik = 0.0;
+    if (lane > k && lane < wm) {
+      lik = A[lane * kLda + k] * inv;
+      A[lane * kLda + k] = lik;
+    }
+    if (lane == k) {
+      A[k * kLda + k] = dkk;
+      invd[k] = inv;
+    }
+    for (int j = k + 1; j < wm; ++j) {
+      const double ljk = __shfl_sync(0xffffffffu, lik, j);
+      if (lane >= j && lane < wm) A[lane * kLda + j] -= lik * ljk;
     }
     __syncwarp();
   }
-  // forward substitution L z = rhs (shared by every window)
-  if (lane < wm) y[lane] = rhs[lane];
-  __syncwarp();
+  // forward substitution L z = rhs (shared by every window): lane i keeps z_i
+  double z = lane < wm ? rhs[lane] : 0.0;
   for (int k = 0; k < wm; ++k) {
-    if (lane == 0) y[k] /= A[k * 32 + k];
-    __syncwarp();
-    if (lane > k && lane < wm) y[lane] -= A[lane * 32 + k] * y[k];
-    __syncwarp();
+    const double zk = __shfl_sync(0xffffffffu, z, k) * invd[k];
+    if (lane == k) z = zk;
+    if (lane > k && lane < wm) z -= A[lane * kLda + k] * zk;
   }
 
   double acc[CPL];
@@ -164,26 +168,24 @@ __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
   for (int c = 0; c < CPL; ++c) acc[c] = 0.0;
   for (int wi = 0; wi < a.n_win; ++wi) {
     const int w = a.windows[wi];
-    // back substitution L_w^T a = z_w on the leading w x w block
-    if (lane < w) coef[lane] = y[lane];
-    __syncwarp();
+    // back substitution L_w^T a = z_w on the leading w x w block: lane i keeps a_i
+    double av = lane < w ? z : 0.0;
     for (int k = w - 1; k >= 0; --k) {
-      if (lane == 0) coef[k] /= A[k * 32 + k];
-      __syncwarp();
-      if (lane < k) coef[lane] -= A[k * 32 + lane] * coef[k];
-      __syncwarp();
+      const double ak = __shfl_sync(0xffffffffu, av, k) * invd[k];
+      if (lane == k) av = ak;
+      if (lane < k) av -= A[k * kLda + lane] * ak;
     }
     // weights over the w lags
-    double wgt = lane < w ? coef[lane] : 0.0;
+    double wgt = lane < w ? av : 0.0;
     if (!a.coef_raw) {
       double m = lane < w ? wgt : -INFINITY;
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
-      double e = lane < w ? exp(wgt - m) : 0.0;
-      double z = e;
+      const double e = lane < w ? exp(wgt - m) : 0.0;
+      double zs = e;
 #pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-      wgt = e / z;
+      for (int o = 16; o >= 1; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
+      wgt = e / zs;
     }
     // lag r (q_{t-1-r}) weights the vector one step later, q_{t-r} = hv[r]
     for (int r = 0; r < w; ++r) {
@@ -205,8 +207,7 @@ cudaError_t launch_predict(const PredictArgs& a, cudaStream_t s) {
   const size_t hv_bytes = (((size_t)(a.wmax + 1) * a.head_dim * 4) + 15) / 16 * 16;
   const size_t smem = kWarps * (hv_bytes + kSolveBytes);
   auto kern = a.head_dim == 64 ? predict_kernel<64> : predict_kernel<128>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
   kern<<<grid, kWarps * 32, smem, s>>>(a);
   return cudaGetLastError();
 }

@@ -274,11 +274,7 @@ cudaError_t launch_score_t(const ScoreParams& p, cudaStream_t s) {
   constexpr int STAGES = (12288 / BLOCK_BYTES) > 2 ? (12288 / BLOCK_BYTES) : 2;
   auto kern = score_kernel<KT, D, G, WARPS, STAGES>;
   const size_t smem = (size_t)WARPS * STAGES * BLOCK_BYTES + WARPS * STAGES * 8 + (2 * (size_t)p.batch + 1) * 4;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WARPS * 32, smem);
-  if (e != cudaSuccess) return e;
+  const int per_sm = prepare_kernel((const void*)kern, smem, WARPS * 32);
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
   kern<<<sm_count() * per_sm, WARPS * 32, smem, s>>>(p);
   return cudaGetLastError();

@@ -5,14 +5,17 @@
 //
 // One thread-block cluster of NC CTAs per row; each CTA keeps its segment of the
 // row as 32-bit order keys in shared memory, so the row is read from L2/HBM once.
-// Radix select, 8 bits per pass from the most significant end: every CTA builds a
-// 256-bin histogram of its candidates (warp-aggregated with match/ballot so hot
-// bins cost one shared atomic per warp), the cluster sums the NC histograms
+// NC is chosen so that the whole grid is resident in one wave.  Radix select
+// from the most significant end with digits of 11, 11 and 10 bits: every CTA
+// builds a histogram of its candidates (warp-aggregated with match/ballot, so a
+// hot bin costs one shared atomic per warp), the cluster sums the NC histograms
 // through distributed shared memory, and every CTA picks the same threshold
-// digit.  A pass stops early once the threshold bin holds exactly the number of
-// tokens still needed.  The ascending write-out is a stable compaction: per
-// 512-token tile, ballots give each token its rank among "above threshold" and
-// "at threshold" tokens, with the counts of lower-ranked CTAs added from DSMEM.
+// digit.  Only keys that still match the threshold prefix take part in later
+// passes, and a pass stops the search once the threshold bin holds exactly the
+// number of tokens still needed (for continuous scores: after two passes).  The
+// ascending write-out is a stable compaction: per 512-token tile, ballots give
+// each token its rank among "above threshold" and "at threshold" tokens, with
+// the counts of lower-ranked CTAs added from DSMEM.
 #include <cooperative_groups.h>
 
 #include "asp_common.cuh"
@@ -26,6 +29,8 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kSegMax = 32768;   // keys per CTA (128 KB of shared memory)
+constexpr int kBins = 2048;      // widest digit: 11 bits
+constexpr int kStaticSmem = 2 * kBins * 4 + 1024;
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -33,7 +38,34 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
+// Exclusive scan of one int per thread over the CTA; also returns the total.
+__device__ __forceinline__ int cta_exclusive_scan(int x, int* wsum, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kWarps ? wsum[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kWarps) wsum[lane] = w;
+  }
+  __syncthreads();
+  const int excl = incl - x + (warp > 0 ? wsum[warp - 1] : 0);
+  *total = wsum[kWarps - 1];
+  __syncthreads();
+  return excl;
+}
+
+__global__ void __launch_bounds__(kThreads, 2) select_kernel(SelectArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
   const int nc = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
@@ -42,11 +74,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   const int b = row / a.rows_per_seq;
 
   extern __shared__ uint32_t keys[];
-  __shared__ int hist[2][256];
-  __shared__ int tot[256];
-  __shared__ int wtot[kWarps];
+  __shared__ int hist[2][kBins];
+  __shared__ int wsum[kWarps];
   __shared__ int wg[kWarps], we[kWarps];
-  __shared__ int s_digit, s_above, s_tile_gt, s_tile_eq, s_last_sel;
+  __shared__ int s_digit, s_above, s_bincnt, s_tile_gt, s_tile_eq, s_last_sel;
   __shared__ int s_cnt[2];
 
   int T = a.seq_lens ? a.seq_lens[b] : a.t_max;
@@ -81,10 +112,12 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   uint32_t prefix = 0u, mask = 0u;
   int krem = a.c_units;
 #pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int nb = pass == 2 ? 1024 : 2048;
+    const uint32_t dmask = (uint32_t)nb - 1u;
     int* h = hist[pass & 1];
-    if (tid < 256) h[tid] = 0;
+    for (int i = tid; i < nb; i += kThreads) h[i] = 0;
     __syncthreads();
     for (int base = 0; base < nloc; base += kThreads) {
       const int i = base + tid;
@@ -93,45 +126,52 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
       if (i < nloc) {
         const uint32_t key = keys[i];
         act = (key & mask) == prefix;
-        dig = (key >> shift) & 255u;
+        dig = (key >> shift) & dmask;
       }
-      const uint32_t peers = __match_any_sync(0xffffffffu, act ? dig : 256u + (uint32_t)lane);
-      if (act && lane == __ffs(peers) - 1) atomicAdd(&h[dig], __popc(peers));
+      const uint32_t am = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const uint32_t peers = __match_any_sync(am, dig);
+        if (lane == __ffs(peers) - 1) atomicAdd(&h[dig], __popc(peers));
+      }
     }
     cluster.sync();
-    if (tid < 256) {
-      int t = 0;
-      for (int r = 0; r < nc; ++r) t += cluster.map_shared_rank(h, r)[tid];
-      tot[tid] = t;
-    }
-    __syncthreads();
-    // thread t < 256 takes digit 255 - t: an inclusive scan over t is a suffix sum over digits
-    int x = 0, incl = 0;
-    if (tid < 256) {
-      x = tot[255 - tid];
-      incl = x;
+    // thread t owns digits nb-1-(t*bpt .. t*bpt+bpt-1): thread order is descending digit order
+    const int bpt = nb / kThreads;
+    int v[kBins / kThreads];
+    int local = 0;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+    for (int j = 0; j < kBins / kThreads; ++j) {
+      v[j] = 0;
+      if (j < bpt) {
+        const int d = nb - 1 - (tid * bpt + j);
+        int sum = 0;
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+          if (r < nc) sum += cluster.map_shared_rank(h, r)[d];
+        v[j] = sum;
+        local += sum;
       }
-      if (lane == 31) wtot[warp] = incl;
     }
-    __syncthreads();
-    if (tid < 256) {
-      for (int w = 0; w < warp; ++w) incl += wtot[w];
-      const int above = incl - x;
-      if (above < krem && krem <= incl) {
-        s_digit = 255 - tid;
-        s_above = above;
+    int total;
+    const int excl = cta_exclusive_scan(local, wsum, &total);
+    if (excl < krem && krem <= excl + local) {
+      int run = excl;
+      for (int j = 0; j < bpt; ++j) {
+        if (run + v[j] >= krem) {
+          s_digit = nb - 1 - (tid * bpt + j);
+          s_above = run;
+          s_bincnt = v[j];
+          break;
+        }
+        run += v[j];
       }
     }
     __syncthreads();
     const int digit = s_digit;
     krem -= s_above;
     prefix |= (uint32_t)digit << shift;
-    mask |= 255u << shift;
-    const bool done = tot[digit] == krem;
+    mask |= dmask << shift;
+    const bool done = s_bincnt == krem;
     __syncthreads();
     if (done) break;
   }
@@ -225,11 +265,22 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   cluster.sync();   // keep this CTA's shared memory alive until the cluster is done reading it
 }
 
+// Cluster size: the largest NC whose grid (rows * NC CTAs) is resident in one
+// wave; if none is, the smallest NC whose segment fits in shared memory.
 int pick_cluster(int rows, int len_max) {
-  const int target = 2 * sm_count();
-  int nc = 1;
-  while (nc < 8 && ((len_max + nc - 1) / nc > kSegMax || rows * nc < target)) nc *= 2;
-  return nc;
+  const int sms = sm_count();
+  int best = 0;
+  for (int nc = 1; nc <= 8; nc *= 2) {
+    const int seg = (len_max + nc - 1) / nc;
+    if (seg > kSegMax) continue;
+    const int smem = seg * 4 + kStaticSmem;
+    int per_sm = (227 * 1024) / smem;
+    per_sm = per_sm > 2 ? 2 : per_sm;
+    if ((long)rows * nc <= (long)sms * per_sm) best = nc;
+    else if (!best) best = -nc;   // remembers the smallest fitting NC
+  }
+  if (best > 0) return best;
+  return best < 0 ? -best : 8;
 }
 
 }  // namespace
@@ -244,8 +295,7 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   const int nc = pick_cluster(a.n_rows, len_max);
   const int seg_max = (len_max + nc - 1) / nc;
   const size_t smem = (size_t)(seg_max > 0 ? seg_max : 1) * 4;
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  if (prepare_kernel((const void*)select_kernel, smem, kThreads) < 1) return cudaErrorInvalidConfiguration;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nc, a.n_rows, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
