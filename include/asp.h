@@ -205,6 +205,30 @@ ASP_API size_t asp_attend_workspace_bytes(int batch, int n_q_heads, int n_kv_hea
                                   int max_tail);
 
 /* ---------------------------------------------------------------------------
+ * Step 4 without a caller-provided workspace.  No counterpart in the paper: this
+ * entry point exists for callers that cannot allocate device memory -- for example
+ * a plug-in inside an engine that owns all device memory and hands the plug-in only
+ * the tensors of the call, or a latency-critical decode loop that must not call
+ * cudaMalloc (it can synchronise the device).  It computes exactly what
+ * asp_sparse_attend computes, with the same arguments minus the workspace.
+ * The split-K partials live in one fixed array inside the library, of
+ * ASP_NOALLOC_SCRATCH_BYTES bytes (2 MiB), that every GPU which loads the library
+ * holds until the process exits.  Sizes whose partials would not fit (compare
+ * asp_attend_workspace_bytes) return ASP_ERR_WORKSPACE and enqueue nothing; with
+ * the current split plan the partials stay below 1.3 MB for every valid size.
+ * The first call on a device looks up the array's device address on that device
+ * (the device must be current); make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents; nothing in
+ * it has to start at zero (every partial the merge reads is written earlier in the
+ * same call).  Calls whose kernels overlap on the GPU (different streams without
+ * ordering between them) race on the array and give wrong results. */
+#define ASP_NOALLOC_SCRATCH_BYTES ((size_t)2 << 20)
+ASP_API asp_status asp_sparse_attend_noalloc(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv,
+                                             const int32_t* idx, const int32_t* count, int C,
+                                             const int32_t* tail_begin, int max_tail, void* out, float* lse,
+                                             asp_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * One asynchronous decode step (steps 1-4).
  * Source: abstract, component (2) (KV selection decoupled from the decoding loop
  * and overlapped with the forward computation).  On one GPU the two ranks of the

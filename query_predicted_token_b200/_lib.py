@@ -50,6 +50,8 @@ SIGNATURES = {
     "asp_sparse_attend": (c_int, [c_void_p, c_int, c_int, POINTER(AspKv), c_void_p, c_void_p, c_int, c_void_p, c_int,
                                   c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "asp_attend_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int]),
+    "asp_sparse_attend_noalloc": (c_int, [c_void_p, c_int, c_int, POINTER(AspKv), c_void_p, c_void_p, c_int, c_void_p,
+                                          c_int, c_void_p, c_void_p, c_void_p]),
     "asp_decode_step": (c_int, [POINTER(AspDecodeArgs)]),
     "asp_wait_selection": (c_int, [c_void_p, c_long]),
     "asp_quest_build_meta": (c_int, [POINTER(AspKv), c_int, c_void_p, c_void_p]),
@@ -188,6 +190,16 @@ def sparse_attend(q: torch.Tensor, kv: KV, idx: Optional[torch.Tensor], count: O
                                                         _ptr(count), int(C), _ptr(tail_begin), int(max_tail),
                                                         _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
                                                         _stream(stream)))
+
+
+def sparse_attend_noalloc(q: torch.Tensor, kv: KV, idx: Optional[torch.Tensor], count: Optional[torch.Tensor],
+                          C: int, out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                          tail_begin: Optional[torch.Tensor] = None, max_tail: int = 0, stream=None) -> None:
+    """Step 4 for callers that cannot allocate: the split-K partials go to the
+    library's fixed scratch array instead of a workspace tensor."""
+    _check("asp_sparse_attend_noalloc", lib().asp_sparse_attend_noalloc(
+        _ptr(q), dtype_code(q), q.shape[1], kv.ref, _ptr(idx), _ptr(count), int(C), _ptr(tail_begin),
+        int(max_tail), _ptr(out), _ptr(lse), _stream(stream)))
 
 
 def quest_build_meta(kv: KV, quest_page: int, meta: torch.Tensor, stream=None) -> None:

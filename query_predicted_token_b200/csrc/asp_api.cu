@@ -241,6 +241,23 @@ asp_status asp_sparse_attend(const void* q, asp_dtype q_dtype, int n_q_heads, co
                                         max_tail, out, lse, workspace, plan, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+asp_status asp_sparse_attend_noalloc(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv,
+                                     const int32_t* idx, const int32_t* count, int C, const int32_t* tail_begin,
+                                     int max_tail, void* out, float* lse, asp_stream_t stream) {
+  // Same validation as asp_sparse_attend; the workspace check is satisfied with a
+  // stand-in (never used: the partials go to the library's fixed scratch), and the
+  // plan's workspace size is then checked against that scratch.
+  asp::AttendPlan plan;
+  void* const stand_in = reinterpret_cast<void*>(static_cast<uintptr_t>(256));
+  asp_status st = check_attend(q, q_dtype, n_q_heads, kv, idx, count, C, tail_begin, max_tail, out, stand_in,
+                               ~static_cast<size_t>(0), &plan);
+  if (st != ASP_OK) return st;
+  if (plan.workspace_bytes > ASP_NOALLOC_SCRATCH_BYTES) return ASP_ERR_WORKSPACE;
+  return cuda_status(asp::launch_attend_noalloc(q, q_dtype == ASP_F32, n_q_heads, view_of(kv), idx, count, C,
+                                                tail_begin, max_tail, out, lse, plan,
+                                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
 asp_status asp_decode_step(const asp_decode_args* a) {
   if (!a) return ASP_ERR_INVALID_ARG;
   asp::AttendPlan plan;

@@ -16,6 +16,7 @@
 //    (max, sum, unnormalised output) go to the workspace and a small kernel does
 //    the log-sum-exp merge.
 #include <cfloat>
+#include <mutex>
 
 #include "asp_common.cuh"
 #include "asp_internal.h"
@@ -496,6 +497,42 @@ cudaError_t launch_attend(const void* q, int q_f32, int n_q_heads, const KvView&
   const int G = n_q_heads / kv.n_kv;
   if (kv.kv_f32) return kv.head_dim == 64 ? dispatch_g<float, 64>(G, p, s) : dispatch_g<float, 128>(G, p, s);
   return kv.head_dim == 64 ? dispatch_g<__nv_bfloat16, 64>(G, p, s) : dispatch_g<__nv_bfloat16, 128>(G, p, s);
+}
+
+// Scratch of asp_sparse_attend_noalloc: the split-K partials of one call, for
+// callers that cannot allocate.  File scope, so every device that loads the
+// library holds it for the life of the process.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ASP_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+static cudaError_t noalloc_scratch_address(void** ptr) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_attend_noalloc(const void* q, int q_f32, int n_q_heads, const KvView& kv, const int32_t* idx,
+                                  const int32_t* count, int C, const int32_t* tail_begin, int max_tail, void* out,
+                                  float* lse, const AttendPlan& plan, cudaStream_t s) {
+  if (plan.workspace_bytes > ASP_NOALLOC_SCRATCH_BYTES) return cudaErrorInvalidValue;
+  void* scratch = nullptr;
+  cudaError_t e = noalloc_scratch_address(&scratch);
+  if (e != cudaSuccess) return e;
+  return launch_attend(q, q_f32, n_q_heads, kv, idx, count, C, tail_begin, max_tail, out, lse, scratch, plan, s);
 }
 
 ASP_STATUS_READER(read_status_attend)

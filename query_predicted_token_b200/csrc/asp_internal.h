@@ -86,6 +86,12 @@ cudaError_t launch_attend(const void* q, int q_f32, int n_q_heads, const KvView&
                           const int32_t* count, int C, const int32_t* tail_begin, int max_tail, void* out,
                           float* lse, void* workspace, const AttendPlan& plan, cudaStream_t s);
 
+// Launches step 4 with its split-K partials in the library's fixed scratch array
+// (asp_sparse_attend_noalloc); `plan.workspace_bytes` must fit in it.
+cudaError_t launch_attend_noalloc(const void* q, int q_f32, int n_q_heads, const KvView& kv, const int32_t* idx,
+                                  const int32_t* count, int C, const int32_t* tail_begin, int max_tail, void* out,
+                                  float* lse, const AttendPlan& plan, cudaStream_t s);
+
 // ---- comparison path ----------------------------------------------------------
 cudaError_t launch_quest_meta(const KvView& kv, int quest_page, void* meta, cudaStream_t s);
 cudaError_t launch_quest_score(const void* q, int q_f32, int n_q_heads, const KvView& kv, const void* meta,
