@@ -73,7 +73,7 @@ typedef enum {
 typedef enum { ASP_F32 = 0, ASP_BF16 = 1 } asp_dtype;
 
 /* How the ridge coefficients of one window become weights (softmax is the
- * method's "softmax-normalized" reading; RAW keeps the coefficients). */
+ * method's softmax normalisation; RAW keeps the coefficients). */
 typedef enum { ASP_COEF_SOFTMAX = 0, ASP_COEF_RAW = 1 } asp_coef_mode;
 
 /* Device status word bits (asp_device_status). */

@@ -3,9 +3,10 @@
 Only tests/, __graft_entry__.smoke() and bench.py's CPU arms may use this.
 
 Pages: the prediction only decides *which* tokens are attended; the decode
-step itself attends over the selected tokens ("attend to the same tokens",
-repro card, "Key finding ..."; "query-aware sparsity without waiting in the
-decoding loop", abstract).  Readings:
+step itself attends over the selected tokens, the same set a page-level
+method would attend at the same budget (repro card, "Key finding ..."), and
+the query-aware sparsity no longer waits inside the decoding loop (abstract).
+Readings:
 
 A1  the attention uses the true current query q_t, not the prediction.
 A2  tokens appended after the selection snapshot, [tail_begin, T_b), are

@@ -2,12 +2,12 @@
 
 Only tests/, __graft_entry__.smoke() and bench.py's CPU arms may use this.
 
-What the pages say: the next query state is predicted "from a short window of
-recent queries" by a light-weight temporal-regressive module (abstract,
-component (1)); the fit is a "softmax-normalized ridge regression with
-multi-window average pooling" (summary, "Problem"/"Approach"); the
-reproduction fits it "one-step-ahead" on a "recent-16-window" (repro card,
-claim C5).  No equation is printed, so the steps below are this reading:
+What the pages say: a light-weight temporal-regressive module predicts the
+next query state from the few most recent queries (abstract, component (1));
+the fit is a ridge regression whose coefficients are normalised by a softmax,
+pooled by averaging over several window lengths (summary, "Approach"); the
+reproduction fits it one step ahead on a window of the last 16 queries (repro
+card, claim C5).  No equation is printed, so the steps below are this reading:
 
 R1  one regression per query head; the samples are the d channels and the
     features are the w lagged query vectors of that head.
@@ -18,10 +18,10 @@ R2  the history holds W+1 vectors q_{t-W} .. q_t (oldest first).  For a
             = (X_w X_w^T + lam I)^{-1} X_w y          (a w x w SPD system).
     The one-step-ahead prediction applies coefficient i to the vector one step
     later:  qhat^(w) = sum_i alpha_{w,i} q_{t-w+i}.
-R3  "softmax-normalized": alpha_w = softmax(a_w) over the w coefficients
+R3  softmax normalisation: alpha_w = softmax(a_w) over the w coefficients
     (temperature 1).  The raw coefficients (alpha = a) are kept as a switch.
 R4  lam is added to the diagonal unscaled.
-R5  "multi-window average pooling": qhat = mean over the windows in Omega of
+R5  multi-window average pooling: qhat = mean over the windows in Omega of
     qhat^(w).
 
 Pins (tests/test_oracle_predict.py): the ridge solve against an augmented

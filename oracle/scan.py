@@ -3,8 +3,8 @@
 Only tests/, __graft_entry__.smoke() and bench.py's CPU arms may use this.
 
 Pages: token-level, query-aware KV selection replaces page-level filtering
-(abstract; summary, "Problem"); the budget is "2k selected tokens" (summary,
-"Key results"; repro card, "Key finding ...": "at C=2k tokens").  The targets
+(abstract; summary, "Problem"); the budget is about two thousand selected
+tokens (summary, "Key results"; repro card, "Key finding ...").  The targets
 are Qwen3 models, whose attention groups G = Hq / Hkv query heads on one KV
 head (summary, "Key results").  Readings:
 
