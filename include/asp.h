@@ -204,6 +204,12 @@ ASP_API asp_status asp_sparse_attend(const void* q, asp_dtype q_dtype, int n_q_h
 ASP_API size_t asp_attend_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C,
                                   int max_tail);
 
+/* Bytes of workspace asp_decode_step needs (attention partials plus the
+ * selection's first-digit histogram, which the key scan builds); a pure function
+ * of its arguments, 0 for invalid sizes. */
+ASP_API size_t asp_decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C,
+                                          int max_tail);
+
 /* ---------------------------------------------------------------------------
  * Step 4 without a caller-provided workspace.  No counterpart in the paper: this
  * entry point exists for callers that cannot allocate device memory -- for example
@@ -240,7 +246,8 @@ ASP_API asp_status asp_sparse_attend_noalloc(const void* q, asp_dtype q_dtype, i
  *            then records ev_sel_done.
  * The caller swaps idx_cur/idx_next (and count_*) between steps, advances
  * ring_start by one, and must not reuse q_t, qpred, scores or idx_next before
- * ev_sel_done completes.  timing: NULL, or 8 events recorded around the kernels
+ * ev_sel_done completes.  workspace: at least asp_decode_workspace_bytes(...)
+ * bytes, 256-byte aligned, no initialisation needed (ASP_ERR_WORKSPACE otherwise).  timing: NULL, or 8 events recorded around the kernels
  * (begin/end of predict, score, select on s_side; attend on s_main) for profiling. */
 typedef struct {
   const void* q_t;              /* device [batch, n_q_heads, head_dim] */

@@ -50,6 +50,7 @@ SIGNATURES = {
     "asp_sparse_attend": (c_int, [c_void_p, c_int, c_int, POINTER(AspKv), c_void_p, c_void_p, c_int, c_void_p, c_int,
                                   c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "asp_attend_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int]),
+    "asp_decode_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int]),
     "asp_sparse_attend_noalloc": (c_int, [c_void_p, c_int, c_int, POINTER(AspKv), c_void_p, c_void_p, c_int, c_void_p,
                                           c_int, c_void_p, c_void_p, c_void_p]),
     "asp_decode_step": (c_int, [POINTER(AspDecodeArgs)]),
@@ -259,7 +260,7 @@ class DecodeState:
         self.idx = [torch.full((B, Hkv, C), -1, dtype=torch.int32, device=dev) for _ in range(2)]
         self.count = [torch.zeros(B, Hkv, dtype=torch.int32, device=dev) for _ in range(2)]
         self.cur = 0
-        ws = attend_workspace_bytes(B, n_q_heads, Hkv, d, C, max_tail if tail_begin is not None else 0)
+        ws = int(lib().asp_decode_workspace_bytes(B, n_q_heads, Hkv, d, C, max_tail if tail_begin is not None else 0))
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
         self.s_main = s_main or torch.cuda.current_stream()
         self.s_side = s_side or torch.cuda.Stream()

@@ -120,9 +120,18 @@ asp_status check_pred(const asp_pred_cfg* cfg, int ring_start) {
 
 asp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ASP_OK : ASP_ERR_CUDA; }
 
+// asp_decode_step's workspace: the attention's split-K partials, then (256-byte
+// aligned) the key-score histogram [batch * n_kv, 2048] int32 of the selection.
+size_t decode_hist_offset(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail) {
+  const size_t att = asp::attend_plan(batch, n_q_heads, n_kv_heads, head_dim, C, max_tail).workspace_bytes;
+  return ((att + 255) / 256) * 256;
+}
+
 asp::PredictArgs predict_args(float* qhist, int ring_start, const void* q_new, asp_dtype q_new_dtype, int batch,
                               int n_q_heads, int head_dim, const asp_pred_cfg* cfg, float* qpred) {
   asp::PredictArgs a;
+  a.zero = nullptr;
+  a.zero_words = 0;
   a.qhist = qhist;
   a.ring_start = ring_start;
   a.q_new = q_new;
@@ -221,7 +230,15 @@ asp_status asp_select_topk(const float* scores, const int32_t* seq_lens, int bat
   a.expand = 1;
   a.idx = idx;
   a.count = count;
+  a.hist0 = nullptr;
   return cuda_status(asp::launch_select(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t asp_decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail) {
+  if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || C < 1 || max_tail < 0) return 0;
+  if (head_dim != 64 && head_dim != 128) return 0;
+  return decode_hist_offset(batch, n_q_heads, n_kv_heads, head_dim, C, max_tail) +
+         (size_t)batch * n_kv_heads * asp::kTopBins * 4;
 }
 
 size_t asp_attend_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail) {
@@ -265,6 +282,13 @@ asp_status asp_decode_step(const asp_decode_args* a) {
                                a->max_tail, a->out, a->workspace, a->workspace_bytes, &plan);
   if (st != ASP_OK) return st;
   if (a->C < 1 || !a->qhist || !a->qpred || !a->scores || !a->idx_next || !a->count_next) return ASP_ERR_INVALID_ARG;
+  const int mt = a->tail_begin ? a->max_tail : 0;
+  const size_t hist_off = decode_hist_offset(a->kv->batch, a->n_q_heads, a->kv->n_kv_heads, a->kv->head_dim, a->C, mt);
+  const size_t hist_words = (size_t)a->kv->batch * a->kv->n_kv_heads * asp::kTopBins;
+  if (!a->workspace || a->workspace_bytes < hist_off + hist_words * 4 ||
+      (reinterpret_cast<uintptr_t>(a->workspace) & 255))
+    return ASP_ERR_WORKSPACE;
+  int32_t* hist = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(a->workspace) + hist_off);
   if (!a->ev_fork || !a->ev_sel_done) return ASP_ERR_INVALID_ARG;
   st = check_pred(a->pred, a->ring_start);
   if (st != ASP_OK) return st;
@@ -286,13 +310,15 @@ asp_status asp_decode_step(const asp_decode_args* a) {
   // side stream: selection for the next step
   if (e == cudaSuccess) e = mark(0, ss);
   if (e == cudaSuccess) {
-    const asp::PredictArgs pa = predict_args(a->qhist, a->ring_start, a->q_t, a->q_dtype, B, a->n_q_heads,
-                                             a->kv->head_dim, a->pred, a->qpred);
+    asp::PredictArgs pa = predict_args(a->qhist, a->ring_start, a->q_t, a->q_dtype, B, a->n_q_heads,
+                                       a->kv->head_dim, a->pred, a->qpred);
+    pa.zero = hist;   // the score kernel accumulates the selection's first histogram here
+    pa.zero_words = hist_words;
     e = asp::launch_predict(pa, ss);
   }
   if (e == cudaSuccess) e = mark(1, ss);
   if (e == cudaSuccess) e = mark(2, ss);
-  if (e == cudaSuccess) e = asp::launch_score(a->qpred, a->n_q_heads, kv, a->scores, ss);
+  if (e == cudaSuccess) e = asp::launch_score(a->qpred, a->n_q_heads, kv, a->scores, ss, hist);
   if (e == cudaSuccess) e = mark(3, ss);
   if (e == cudaSuccess) e = mark(4, ss);
   if (e == cudaSuccess) {
@@ -307,6 +333,7 @@ asp_status asp_decode_step(const asp_decode_args* a) {
     sa.expand = 1;
     sa.idx = a->idx_next;
     sa.count = a->count_next;
+    sa.hist0 = hist;
     e = asp::launch_select(sa, ss);
   }
   if (e == cudaSuccess) e = mark(5, ss);
@@ -370,6 +397,7 @@ asp_status asp_quest_select(const void* q, asp_dtype q_dtype, int n_q_heads, con
   sa.expand = quest_page;
   sa.idx = idx;
   sa.count = count;
+  sa.hist0 = nullptr;
   return cuda_status(asp::launch_select(sa, s));
 }
 

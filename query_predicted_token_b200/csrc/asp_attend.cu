@@ -136,7 +136,14 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(AttParams p) {
   // tile t of this warp covers rows r0 + (warp + t * kWarps) * kTile + [0, 16)
   const int my_tiles = n_tiles > warp ? (n_tiles - warp + kWarps - 1) / kWarps : 0;
 
-  auto issue = [&](int t, int slot) -> uint32_t {
+  // Row source of this lane for tile t (lanes 0-15: K rows, 16-31: V rows).  The
+  // index and page-table loads of the next tile are issued one tile ahead, so
+  // their latency hides behind the current tile's compute.
+  struct RowSrc {
+    const uint8_t* src;
+    bool valid;
+  };
+  auto resolve = [&](int t) -> RowSrc {
     const int rr = lane & 15;
     const bool isv = lane >= 16;
     const int r = r0 + (warp + t * kWarps) * kTile + rr;
@@ -170,9 +177,16 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(AttParams p) {
         }
       }
     }
-    const uint32_t vm = __ballot_sync(0xffffffffu, valid) & 0xffffu;
+    return RowSrc{src, valid};
+  };
+  // Gathers one tile into a stage: one bulk copy per valid row, rows with no
+  // source zero-filled; returns the tile's valid-row mask.
+  auto issue = [&](const RowSrc& rs, int slot) -> uint32_t {
+    const int rr = lane & 15;
+    const bool isv = lane >= 16;
+    const uint32_t vm = __ballot_sync(0xffffffffu, rs.valid) & 0xffffu;
     uint8_t* dst = wbuf + slot * TILE_BYTES + (isv ? kTile * ROW_BYTES : 0) + rr * ROW_BYTES;
-    if (!valid) {
+    if (!rs.valid) {
 #pragma unroll
       for (int c = 0; c < ROW_BYTES / 16; ++c) reinterpret_cast<uint4*>(dst)[c] = make_uint4(0, 0, 0, 0);
     }
@@ -180,7 +194,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(AttParams p) {
     __syncwarp();
     if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)__popc(vm) * 2u * ROW_BYTES);
     __syncwarp();
-    if (valid) bulk_g2s(dst, src, ROW_BYTES, &bars[slot]);
+    if (rs.valid) bulk_g2s(dst, rs.src, ROW_BYTES, &bars[slot]);
     return vm;
   };
 
@@ -196,9 +210,10 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(AttParams p) {
   int issued = 0;
 #pragma unroll 1
   for (int s = 0; s < STAGES && s < my_tiles; ++s) {
-    vmask[s] = issue(s, s);
+    vmask[s] = issue(resolve(s), s);
     ++issued;
   }
+  RowSrc next = issued < my_tiles ? resolve(issued) : RowSrc{nullptr, false};
 
   int consumed = 0;
   bool ok = true;
@@ -309,8 +324,9 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(AttParams p) {
     }
     __syncwarp();
     if (issued < my_tiles) {
-      vmask[slot] = issue(issued, slot);
+      vmask[slot] = issue(next, slot);
       ++issued;
+      if (issued < my_tiles) next = resolve(issued);
     }
   }
   if (!ok) {

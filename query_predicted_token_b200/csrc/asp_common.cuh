@@ -113,6 +113,19 @@ __device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32
       : "memory");
 }
 
+// ---- selection keys ---------------------------------------------------------
+
+// 32-bit key whose unsigned order is the IEEE order of the score (-0.0 == +0.0).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Width of the first radix digit of the selection (the key's top 11 bits).
+constexpr int kTopBins = 2048;
+constexpr int kTopShift = 21;
+
 // ---- element conversion -----------------------------------------------------
 
 // Two bf16 packed in a 32-bit word -> (low, high) as fp32 (exact).

@@ -28,6 +28,8 @@ cudaError_t read_status_quest(cudaStream_t s, int* bits);
 
 // ---- step 1 -----------------------------------------------------------------
 struct PredictArgs {
+  int32_t* zero;          // optional buffer the kernel clears first (next step's key histogram)
+  size_t zero_words;
   float* qhist;
   int ring_start;
   const void* q_new;      // may be null
@@ -54,7 +56,10 @@ struct KvView {
   const int32_t* page_table;
   const int32_t* seq_lens;   // may be null (all t_max)
 };
-cudaError_t launch_score(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s);
+// hist: optional [batch * n_kv, 2048] int32 counts of the scores' top 11 key bits
+// (must be zero on entry); the selection then skips its own first pass.
+cudaError_t launch_score(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s,
+                         int32_t* hist = nullptr);
 
 // ---- step 3 -----------------------------------------------------------------
 // Selects `c_units` units per row out of ceil(T_b / expand) scores (row stride
@@ -71,6 +76,7 @@ struct SelectArgs {
   int expand;
   int32_t* idx;
   int32_t* count;
+  const int32_t* hist0;      // optional first-pass histogram [n_rows, 2048] (expand == 1 only)
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
 bool select_supported(int t_max, int expand);

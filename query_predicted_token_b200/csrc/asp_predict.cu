@@ -7,15 +7,20 @@
 // One warp per query head; the history is tiny (17 x 128 fp32 for W = 16), so
 // the kernel is latency-bound and the work is arranged to keep the dependency
 // chains short:
+//  * every lane loads its 16-byte slice of every history vector up front (all
+//    loads in flight at once) and keeps them in registers;
 //  * the lags are ordered newest first (r = 0 is q_{t-1}), which makes every
 //    window's system the *leading* w x w block of one matrix.  A Cholesky
 //    factor's leading block is the factor of the leading block, and the forward
 //    substitution of a leading block is the leading part of the full one, so a
 //    single factorisation and forward solve serve all windows; only the back
 //    substitution is per window;
-//  * Gram and right-hand side in fp64 (products of fp32 values are exact in
-//    fp64), chunked over 32 (i, j) pairs with a warp reduce-scatter;
-//  * the Cholesky is warp-parallel (right-looking: lane i updates row i).
+//  * Gram and right-hand side in fp32 (the lane's partial dot products, summed
+//    over the warp with a 32-wide reduce-scatter), the Cholesky and both
+//    substitutions in fp64 (the lag Gram's condition number is ~1e3 on AR(1)
+//    histories; fp64 keeps the coefficients' error far below the output bound);
+//  * the Cholesky is warp-parallel (pivot computed by every lane, column
+//    broadcast by shuffles, lane i updates row i).
 #include "asp_common.cuh"
 #include "asp_internal.h"
 
@@ -48,93 +53,113 @@ struct ReduceScatterD {
   }
 };
 
-template <int D>
+// Stores the reduced pair `q` (lane's pair of a round) into the solve arrays:
+// pairs (i >= 1, j >= 1) are lag-Gram entries, pairs (i >= 1, 0) the right-hand side.
+__device__ __forceinline__ void store_pair(int q, float val, int wmax, double lam, double* A, double* rhs) {
+  int qi = (int)((sqrtf(8.f * q + 1.f) - 1.f) * 0.5f);
+  while (qi * (qi + 1) / 2 > q) --qi;
+  while ((qi + 1) * (qi + 2) / 2 <= q) ++qi;
+  const int qj = q - qi * (qi + 1) / 2;
+  if (qi >= 1 && qi <= wmax) {
+    if (qj >= 1) A[(qi - 1) * kLda + (qj - 1)] = (double)val + (qi == qj ? lam : 0.0);
+    else rhs[qi - 1] = (double)val;
+  }
+}
+
+// Compile-time walk over the pairs (I, J), J <= I, P = I (I + 1) / 2 + J, so that
+// every register of the history is addressed statically (rows outer, columns
+// inner keeps the template recursion shallow).
+template <int NV, int CPL, int I, int J>
+struct GramCol {
+  __device__ __forceinline__ static void run(const float (&h)[NV][CPL], float (&part)[32], int lane, int wmax,
+                                             double lam, double* A, double* rhs) {
+    constexpr int NPAIR = NV * (NV + 1) / 2;
+    constexpr int P = I * (I + 1) / 2 + J;
+    float acc = h[I][0] * h[J][0];
+#pragma unroll
+    for (int c = 1; c < CPL; ++c) acc = fmaf(h[I][c], h[J][c], acc);
+    part[P % 32] = acc;
+    if constexpr (P % 32 == 31 || P == NPAIR - 1) {
+#pragma unroll
+      for (int k = P % 32 + 1; k < 32; ++k) part[k] = 0.f;
+      ReduceScatter<32, 16>::run(part, lane);
+      const int q = (P / 32) * 32 + lane;
+      if (q < NPAIR) store_pair(q, part[0], wmax, lam, A, rhs);
+    }
+    if constexpr (J < I) GramCol<NV, CPL, I, J + 1>::run(h, part, lane, wmax, lam, A, rhs);
+  }
+};
+
+template <int NV, int CPL, int I>
+struct GramRows {
+  __device__ __forceinline__ static void run(const float (&h)[NV][CPL], float (&part)[32], int lane, int wmax,
+                                             double lam, double* A, double* rhs) {
+    GramCol<NV, CPL, I, 0>::run(h, part, lane, wmax, lam, A, rhs);
+    if constexpr (I + 1 < NV) GramRows<NV, CPL, I + 1>::run(h, part, lane, wmax, lam, A, rhs);
+  }
+};
+
+template <int D, int NV>
 __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
-  constexpr int CPL = D / 32;   // channels per lane
+  constexpr int CPL = D / 32;   // contiguous channels per lane
   extern __shared__ __align__(16) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head = blockIdx.x * kWarps + warp;
+  if (a.zero) {   // clear the next kernel's histogram (16-byte stores, spread over all warps)
+    const size_t n4 = a.zero_words / 4;
+    int4* z4 = reinterpret_cast<int4*>(a.zero);
+    for (size_t i = (size_t)head * 32 + lane; i < n4; i += (size_t)gridDim.x * kWarps * 32) z4[i] = make_int4(0, 0, 0, 0);
+    for (size_t i = n4 * 4 + (size_t)head * 32 + lane; i < a.zero_words; i += (size_t)gridDim.x * kWarps * 32) a.zero[i] = 0;
+  }
   if (head >= a.n_heads) return;
 
-  const int n = a.wmax + 1;            // vectors used: target + wmax lags
-  const int nslot = a.W + 1;
-  // per-warp shared memory: hv[n][D] fp32, A[wmax][wmax] fp64, rhs[wmax], y[wmax], coef[wmax]
-  const size_t hv_bytes = (((size_t)(a.wmax + 1) * D * 4) + 15) / 16 * 16;
-  uint8_t* base = smem + warp * (hv_bytes + kSolveBytes);
-  float* hv = reinterpret_cast<float*>(base);
-  double* A = reinterpret_cast<double*>(base + hv_bytes);
+  double* A = reinterpret_cast<double*>(smem + warp * kSolveBytes);   // [32][kLda] lag Gram, then L
   double* rhs = A + 32 * kLda;
   double* invd = rhs + 32;
 
+  const int n = a.wmax + 1;   // vectors used: the target and wmax lags
+  const int nslot = a.W + 1;
   float* hist = a.qhist + (size_t)head * nslot * D;
-  // chronological position s (0 = oldest, W = newest) -> ring slot
   const int start = a.q_new ? a.ring_start + 1 : a.ring_start;
-  // hv[0] = q_t (target), hv[1 + r] = q_{t-1-r} for r < wmax
-  for (int v = 0; v < n; ++v) {
-    const int s = a.W - v;   // chronological position of hv[v]
-    const int slot = (start + s) % nslot;
-    for (int c = lane; c < D; c += 32) {
-      float x;
-      if (a.q_new && v == 0) {
-        const size_t off = (size_t)head * D + c;
-        x = a.q_new_f32 ? static_cast<const float*>(a.q_new)[off]
-                        : __bfloat162float(static_cast<const __nv_bfloat16*>(a.q_new)[off]);
-        hist[(size_t)slot * D + c] = x;   // push into the ring (slot == ring_start)
+  // h[v] = q_{t-v}: h[0] is the target q_t, h[1 + r] is lag r (q_{t-1-r})
+  float h[NV][CPL];
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) h[v][c] = 0.f;
+    if (v < n) {
+      const int slot = (start + a.W - v) % nslot;
+      float* src = hist + (size_t)slot * D + lane * CPL;
+      if (v == 0 && a.q_new) {
+        const size_t off = (size_t)head * D + lane * CPL;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c)
+          h[0][c] = a.q_new_f32 ? static_cast<const float*>(a.q_new)[off + c]
+                                : __bfloat162float(static_cast<const __nv_bfloat16*>(a.q_new)[off + c]);
+      } else if constexpr (CPL == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(src);
+        h[v][0] = x.x; h[v][1] = x.y; h[v][2] = x.z; h[v][3] = x.w;
       } else {
-        x = hist[(size_t)slot * D + c];
+        const float2 x = *reinterpret_cast<const float2*>(src);
+        h[v][0] = x.x; h[v][1] = x.y;
       }
-      hv[v * D + c] = x;
     }
+  }
+  if (a.q_new) {   // push q_t into the ring: it replaces the oldest slot (ring_start)
+    float* dst = hist + (size_t)a.ring_start * D + lane * CPL;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) dst[c] = h[0][c];
+  }
+
+  // Gram of the n vectors: pairs (i, j), j <= i < NV, enumerated row by row, 32
+  // per round; after the reduce-scatter lane l holds pair (round base + l).
+  {
+    float part[32];
+    GramRows<NV, CPL, 0>::run(h, part, lane, a.wmax, a.lam, A, rhs);
   }
   __syncwarp();
 
-  // Gram over the lags (newest first) and right-hand side, fp64, 32 pairs per round.
-  // Pairs are enumerated as the lower triangle (i, j), j <= i < wmax, row by row,
-  // followed by the wmax (lag i, target) pairs of the right-hand side.
   const int wm = a.wmax;
-  const int n_lag_pairs = wm * (wm + 1) / 2;
-  const int n_pairs = n_lag_pairs + wm;
-  int ci = 0, cj = 0;   // pair cursor (uniform across the warp)
-  for (int p0 = 0; p0 < n_pairs; p0 += 32) {
-    double vals[32];
-    int si = ci, sj = cj;   // first pair of this round
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const int pi = p0 + k;
-      double acc = 0.0;
-      if (pi < n_pairs) {
-        const int u = (ci < wm) ? 1 + ci : 1 + cj;   // lag row
-        const int v = (ci < wm) ? 1 + cj : 0;        // lag column, or the target
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-          const int ch = lane + 32 * c;
-          acc = fma((double)hv[u * D + ch], (double)hv[v * D + ch], acc);
-        }
-        if (ci < wm) {
-          if (++cj > ci) { ++ci; cj = 0; }
-        } else {
-          ++cj;
-        }
-      }
-      vals[k] = acc;
-    }
-    ReduceScatterD<32, 16>::run(vals, lane);
-    // lane holds pair p0 + lane: step the round's first pair forward by `lane`
-    int ti = si, tj = sj;
-    for (int k = 0; k < lane; ++k) {
-      if (ti < wm) {
-        if (++tj > ti) { ++ti; tj = 0; }
-      } else {
-        ++tj;
-      }
-    }
-    if (p0 + lane < n_pairs) {
-      if (ti < wm) A[ti * kLda + tj] = vals[0] + (ti == tj ? a.lam : 0.0);
-      else rhs[tj] = vals[0];
-    }
-  }
-  __syncwarp();
-
   // Cholesky A = L L^T in place (lower triangle), right-looking.  Every lane
   // computes the pivot; lane i owns row i; column k is broadcast by shuffles.
   for (int k = 0; k < wm; ++k) {
@@ -163,11 +188,14 @@ __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
     if (lane > k && lane < wm) z -= A[lane * kLda + k] * zk;
   }
 
-  double acc[CPL];
+  float acc[CPL];
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) acc[c] = 0.0;
+  for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
   for (int wi = 0; wi < a.n_win; ++wi) {
-    const int w = a.windows[wi];
+    int w = 0;   // a.windows[wi] without a dynamically indexed copy of the parameters
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (k == wi) w = a.windows[k];
     // back substitution L_w^T a = z_w on the leading w x w block: lane i keeps a_i
     double av = lane < w ? z : 0.0;
     for (int k = w - 1; k >= 0; --k) {
@@ -187,29 +215,45 @@ __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
       for (int o = 16; o >= 1; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
       wgt = e / zs;
     }
-    // lag r (q_{t-1-r}) weights the vector one step later, q_{t-r} = hv[r]
-    for (int r = 0; r < w; ++r) {
-      const double wr = __shfl_sync(0xffffffffu, wgt, r);
+    // lag r (q_{t-1-r}) weights the vector one step later, q_{t-r} = h[r]
+    const float wf = (float)wgt;
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) acc[c] = fma(wr, (double)hv[r * D + lane + 32 * c], acc[c]);
+    for (int r = 0; r < NV - 1; ++r) {
+      const float wr = __shfl_sync(0xffffffffu, wf, r);
+      if (r < w) {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) acc[c] = fmaf(wr, h[r][c], acc[c]);
+      }
     }
-    __syncwarp();
   }
-  float* out = a.qpred + (size_t)head * D;
+  float* out = a.qpred + (size_t)head * D + lane * CPL;
+  const float inv_nw = 1.f / (float)a.n_win;
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) out[lane + 32 * c] = (float)(acc[c] / a.n_win);
+  for (int c = 0; c < CPL; ++c) out[c] = acc[c] * inv_nw;
+}
+
+
+template <int D, int NV>
+cudaError_t launch_t(const PredictArgs& a, cudaStream_t s) {
+  const int grid = (a.n_heads + kWarps - 1) / kWarps;
+  const size_t smem = kWarps * kSolveBytes;
+  auto kern = predict_kernel<D, NV>;
+  if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
+  kern<<<grid, kWarps * 32, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const PredictArgs& a, cudaStream_t s) {
+  if (a.wmax + 1 <= 9) return launch_t<D, 9>(a, s);
+  if (a.wmax + 1 <= 17) return launch_t<D, 17>(a, s);
+  return launch_t<D, 33>(a, s);
 }
 
 }  // namespace
 
 cudaError_t launch_predict(const PredictArgs& a, cudaStream_t s) {
-  const int grid = (a.n_heads + kWarps - 1) / kWarps;
-  const size_t hv_bytes = (((size_t)(a.wmax + 1) * a.head_dim * 4) + 15) / 16 * 16;
-  const size_t smem = kWarps * (hv_bytes + kSolveBytes);
-  auto kern = a.head_dim == 64 ? predict_kernel<64> : predict_kernel<128>;
-  if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
-  kern<<<grid, kWarps * 32, smem, s>>>(a);
-  return cudaGetLastError();
+  return a.head_dim == 64 ? launch_d<64>(a, s) : launch_d<128>(a, s);
 }
 
 ASP_STATUS_READER(read_status_predict)

@@ -32,6 +32,7 @@ struct ScoreParams {
   const int32_t* page_table;
   const int32_t* seq_lens;
   float* scores;
+  int32_t* hist;   // optional per-row histogram of the top 11 key bits
   float scale;
 };
 
@@ -247,10 +248,23 @@ __global__ void __launch_bounds__(WARPS * 32, 1) score_kernel(ScoreParams p) {
 #pragma unroll
       for (int o = 1; o < LPS; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       const int l = lane % LPR;
+      bool has = false;
       if (l % LPS == 0) {
         const int row = (pass * SPP + l / LPS) * RPS + lane / LPR;
         const int j = j0 + row;
-        if (j < cc.T) srow[j] = m;
+        if (j < cc.T) {
+          srow[j] = m;
+          has = true;
+        }
+      }
+      if (p.hist) {   // first radix pass of the selection, fused: count the top key bits
+        const uint32_t dig = order_key(m) >> kTopShift;
+        const uint32_t hm = __ballot_sync(0xffffffffu, has);
+        if (has) {
+          const uint32_t peers = __match_any_sync(hm, dig);
+          if (lane == __ffs(peers) - 1)
+            atomicAdd(p.hist + (size_t)(cc.b * p.n_kv + cc.h) * kTopBins + dig, __popc(peers));
+        }
       }
     }
     __syncwarp();
@@ -293,7 +307,8 @@ cudaError_t dispatch_g(int G, const ScoreParams& p, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_score(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s) {
+cudaError_t launch_score(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s,
+                         int32_t* hist) {
   ScoreParams p;
   p.qpred = qpred;
   p.n_q_heads = n_q_heads;
@@ -307,6 +322,7 @@ cudaError_t launch_score(const float* qpred, int n_q_heads, const KvView& kv, fl
   p.page_table = kv.page_table;
   p.seq_lens = kv.seq_lens;
   p.scores = scores;
+  p.hist = hist;
   p.scale = 1.0f / sqrtf((float)kv.head_dim);
   const int G = n_q_heads / kv.n_kv;
   if (kv.kv_f32) {

@@ -142,6 +142,14 @@ def test_attend_workspace_rules(lib):
     assert st == L.ASP_ERR_INVALID_ARG
 
 
+def test_decode_workspace_holds_the_partials_and_the_histogram(lib):
+    att = lib.asp_attend_workspace_bytes(8, 32, 8, 128, 2048, 0)
+    dec = lib.asp_decode_workspace_bytes(8, 32, 8, 128, 2048, 0)
+    assert dec >= ((att + 255) // 256) * 256 + 8 * 8 * 2048 * 4
+    assert lib.asp_decode_workspace_bytes(8, 32, 8, 96, 2048, 0) == 0
+    assert lib.asp_decode_workspace_bytes(8, 32, 8, 128, 0, 0) == 0
+
+
 def test_workspace_grows_with_the_tail(lib):
     a = lib.asp_attend_workspace_bytes(64, 32, 8, 128, 2048, 0)
     b = lib.asp_attend_workspace_bytes(64, 32, 8, 128, 2048, 4096)
