@@ -410,6 +410,7 @@ asp_status asp_device_status(asp_stream_t stream, int32_t* bits_out) {
   if (e == cudaSuccess) e = asp::read_status_select(s, &v);
   if (e == cudaSuccess) e = asp::read_status_attend(s, &v);
   if (e == cudaSuccess) e = asp::read_status_quest(s, &v);
+  if (e == cudaSuccess) e = asp::read_status_score_tc(s, &v);
   if (bits_out) *bits_out = v;
   if (e != cudaSuccess) return ASP_ERR_CUDA;
   return v ? ASP_ERR_DEVICE : ASP_OK;

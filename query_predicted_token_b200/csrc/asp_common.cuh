@@ -192,6 +192,38 @@ struct ReduceScatter {
   }
 };
 
+// pre[0] = 0, pre[i + 1] = pre[i] + f(i) for i < n; the whole CTA participates.
+template <typename F>
+__device__ void cta_prefix_sum(int n, int* pre, F f, int* scratch) {
+  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, wid = tid >> 5, nw = nt >> 5;
+  int carry = 0;
+  if (tid == 0) pre[0] = 0;
+  for (int base = 0; base < n; base += nt) {
+    const int i = base + tid;
+    int x = i < n ? f(i) : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) scratch[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      int w = lane < nw ? scratch[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      if (lane < nw) scratch[lane] = w;
+    }
+    __syncthreads();
+    if (i < n) pre[i + 1] = carry + (wid > 0 ? scratch[wid - 1] : 0) + x;
+    carry += scratch[nw - 1];
+    __syncthreads();
+  }
+}
+
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 }  // namespace asp

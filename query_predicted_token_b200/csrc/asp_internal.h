@@ -25,6 +25,7 @@ cudaError_t read_status_score(cudaStream_t s, int* bits);
 cudaError_t read_status_select(cudaStream_t s, int* bits);
 cudaError_t read_status_attend(cudaStream_t s, int* bits);
 cudaError_t read_status_quest(cudaStream_t s, int* bits);
+cudaError_t read_status_score_tc(cudaStream_t s, int* bits);
 
 // ---- step 1 -----------------------------------------------------------------
 struct PredictArgs {
@@ -60,6 +61,12 @@ struct KvView {
 // (must be zero on entry); the selection then skips its own first pass.
 cudaError_t launch_score(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s,
                          int32_t* hist = nullptr);
+
+// Tensor-core key scan (bf16 keys, head_dim 64/128, contiguous or 16-token pages,
+// G in {1,2,4,8}, 16-byte aligned qpred); launch_score uses it when supported.
+bool score_tc_supported(const KvView& kv, int n_q_heads, const float* qpred);
+cudaError_t launch_score_tc(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s,
+                            int32_t* hist);
 
 // ---- step 3 -----------------------------------------------------------------
 // Selects `c_units` units per row out of ceil(T_b / expand) scores (row stride

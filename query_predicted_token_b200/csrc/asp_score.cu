@@ -40,38 +40,6 @@ struct Cursor {
   int b, h, blk, nblk, T;
 };
 
-// pre[0] = 0, pre[i + 1] = pre[i] + f(i) for i < n; the whole CTA participates.
-template <typename F>
-__device__ void cta_prefix_sum(int n, int* pre, F f, int* scratch) {
-  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, wid = tid >> 5, nw = nt >> 5;
-  int carry = 0;
-  if (tid == 0) pre[0] = 0;
-  for (int base = 0; base < n; base += nt) {
-    const int i = base + tid;
-    int x = i < n ? f(i) : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) scratch[wid] = x;
-    __syncthreads();
-    if (wid == 0) {
-      int w = lane < nw ? scratch[lane] : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, w, o);
-        if (lane >= o) w += y;
-      }
-      if (lane < nw) scratch[lane] = w;
-    }
-    __syncthreads();
-    if (i < n) pre[i + 1] = carry + (wid > 0 ? scratch[wid - 1] : 0) + x;
-    carry += scratch[nw - 1];
-    __syncthreads();
-  }
-}
-
 template <typename KT, int D, int G, int WARPS, int STAGES>
 __global__ void __launch_bounds__(WARPS * 32, 1) score_kernel(ScoreParams p) {
   using E = Elem<KT>;
@@ -309,6 +277,7 @@ cudaError_t dispatch_g(int G, const ScoreParams& p, cudaStream_t s) {
 
 cudaError_t launch_score(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s,
                          int32_t* hist) {
+  if (score_tc_supported(kv, n_q_heads, qpred)) return launch_score_tc(qpred, n_q_heads, kv, scores, s, hist);
   ScoreParams p;
   p.qpred = qpred;
   p.n_q_heads = n_q_heads;

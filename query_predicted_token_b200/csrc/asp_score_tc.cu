@@ -1,0 +1,416 @@
+// asp_score_tc.cu -- step 2 on the 5th-generation tensor cores (bf16 keys).
+//
+// scores[b, h, j] = max_g (qpred[b, h*G+g] . k[b, h, j]) / sqrt(d) as the
+// contraction S = K Q^T with K a 128-token x d tile (MMA M = 128) and Q the
+// group's G predicted queries.  q_hat is fp32: each scaled query is split into
+// bf16 hi = rn(q) and lo = rn(q - hi) (residual below 2^-17 |q|), both become
+// rows of the B operand (N = 2G padded to 16), and the epilogue adds the two
+// columns of each head -- bf16 x bf16 products are exact in the fp32
+// accumulator, so the split keeps fp32-class accuracy at tensor-core rate.
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0     producer: 2-D TMA loads (128-byte swizzle) of each 128-token key
+//              tile into a 4-stage ring, plus the tile's Q rows written in the
+//              same swizzled K-major layout;
+//   warp 1     allocates 32 TMEM columns and issues tcgen05.mma (M128 N16 K16,
+//              fp32 accumulate) into one of two TMEM accumulators, committing to
+//              the stage's "empty" and the accumulator's "full" barriers;
+//   warps 2-5  epilogue: tcgen05.ld of their 32 TMEM lanes (one token each),
+//              hi + lo per head, max over the group, coalesced store, and the
+//              selection's first-digit histogram.
+// Every barrier wait is bounded (ASP_DEV_WAIT_LIMIT).  The contiguous cache is
+// one 2-D tensor [B*Hkv*t_max, d]; the paged cache [n_pages*Hkv*16, d] with one
+// 16-row box per page.
+#include <cuda.h>
+
+#include "asp_common.cuh"
+#include "asp_internal.h"
+
+namespace asp {
+namespace {
+
+constexpr int kTileT = 128;    // tokens per tile = MMA M
+constexpr int kN = 16;         // MMA N: rows (hi, lo) of the group's queries, padded
+constexpr int kStages = 4;
+constexpr int kThreadsTC = 192;
+constexpr uint32_t kTmemCols = 32;   // two 16-column fp32 accumulators
+// instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major, N, M
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kN >> 3) << 17) |
+                            ((uint32_t)(kTileT >> 4) << 24);
+
+struct TcParams {
+  const float* qpred;
+  int n_q_heads, G;   // G is also the kernel's template argument
+  int batch, n_kv, t_max, page_size, max_pages, n_pages;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  float* scores;
+  int32_t* hist;
+  float scale;
+};
+
+struct TileCursor {
+  int b, h, tile, ntile, T;
+};
+
+// shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo_elem, float hi_elem) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                                 TcParams p) {
+  constexpr int HALVES = D / 64;                      // 64-channel (128-byte) swizzle columns
+  constexpr int KBYTES = kTileT * D * 2;              // one key tile
+  constexpr int QBYTES = HALVES * kN * 128;           // the tile's B operand
+  constexpr int STAGE = KBYTES + QBYTES;              // multiple of 1024
+  constexpr int KSTEPS = D / 16;
+  constexpr int QCH = HALVES * kN * 8 / 32;           // 16-byte Q chunks per producer lane
+  static_assert(STAGE % 1024 == 0, "stage alignment");
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t s_tmem;
+  __shared__ int scratch[33];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * STAGE);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  int* pre = reinterpret_cast<int*>(tempty + 2);
+  int* lens = pre + p.batch + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  for (int b = threadIdx.x; b < p.batch; b += blockDim.x) {
+    int t = p.seq_lens ? p.seq_lens[b] : p.t_max;
+    lens[b] = t < 0 ? 0 : (t > p.t_max ? p.t_max : t);
+  }
+  __syncthreads();
+  cta_prefix_sum(p.batch, pre, [&](int b) { return ((lens[b] + kTileT - 1) / kTileT) * p.n_kv; }, scratch);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init_fence();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  const int total = pre[p.batch];
+  const int chunk = (total + gridDim.x - 1) / gridDim.x;
+  const int t0 = min(total, (int)blockIdx.x * chunk);
+  const int t1 = min(total, t0 + chunk);
+  const int n_my = t1 - t0;
+
+  auto locate = [&](int i, TileCursor& c) {
+    int lo = 0, hi = p.batch;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pre[mid] <= i) lo = mid; else hi = mid;
+    }
+    c.b = lo;
+    c.T = lens[lo];
+    c.ntile = (pre[lo + 1] - pre[lo]) / p.n_kv;
+    const int r = i - pre[lo];
+    c.h = r / c.ntile;
+    c.tile = r - c.h * c.ntile;
+  };
+  auto advance = [&](TileCursor& c) {
+    if (++c.tile == c.ntile) {
+      c.tile = 0;
+      if (++c.h == p.n_kv) {
+        c.h = 0;
+        do { ++c.b; } while (c.b < p.batch && pre[c.b + 1] == pre[c.b]);
+        if (c.b < p.batch) {
+          c.T = lens[c.b];
+          c.ntile = (pre[c.b + 1] - pre[c.b]) / p.n_kv;
+        }
+      }
+    }
+  };
+
+  if (n_my > 0 && warp == 0) {
+    // ------------------------------------------------------------ producer
+    const uint64_t policy = l2_evict_first_policy();
+    TileCursor c;
+    locate(t0, c);
+    int qb = -1, qh = -1;
+    uint4 qreg[QCH];
+    int issued = 0, done_ok = 1;
+    for (int k = 0; k < n_my; ++k) {
+      const int s = k % kStages;
+      const uint32_t ph = (uint32_t)(k / kStages) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u))) {
+        done_ok = 0;
+        break;
+      }
+      if (c.b != qb || c.h != qh) {   // the group's queries as bf16 hi / lo rows
+        qb = c.b;
+        qh = c.h;
+#pragma unroll
+        for (int m = 0; m < QCH; ++m) {
+          const int cid = lane + 32 * m;   // chunk: half, row, 8-channel column
+          const int half = cid / (kN * 8), r = (cid / 8) % kN, col = cid % 8;
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = 0.f;
+          const int g = r < G ? r : r - G;
+          if (r < 2 * G) {
+            const float* src = p.qpred + ((size_t)(c.b * p.n_q_heads + c.h * G + g)) * D + half * 64 + col * 8;
+            const float4 a0 = *reinterpret_cast<const float4*>(src);
+            const float4 a1 = *reinterpret_cast<const float4*>(src + 4);
+            const float v[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float q = v[e] * p.scale;
+              const float hi = __bfloat162float(__float2bfloat16_rn(q));
+              x[e] = r < G ? hi : q - hi;
+            }
+          }
+          qreg[m] = make_uint4(bf16x2_bits(x[0], x[1]), bf16x2_bits(x[2], x[3]), bf16x2_bits(x[4], x[5]),
+                               bf16x2_bits(x[6], x[7]));
+        }
+      }
+      uint8_t* st = smem + s * STAGE;
+#pragma unroll
+      for (int m = 0; m < QCH; ++m) {
+        const int cid = lane + 32 * m;
+        const int half = cid / (kN * 8), r = (cid / 8) % kN, col = cid % 8;
+        *reinterpret_cast<uint4*>(st + KBYTES + half * (kN * 128) + r * 128 + ((col ^ (r & 7)) << 4)) = qreg[m];
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], KBYTES);
+      __syncwarp();
+      const uint32_t sdst = sbase + s * STAGE;
+      if (p.page_size == 0) {
+        if (lane < HALVES) {
+          const int y = (c.b * p.n_kv + c.h) * p.t_max + c.tile * kTileT;
+          tma_load_2d(sdst + lane * (kTileT * 128), &kmap, lane * 64, y, &full[s], policy);
+        }
+      } else if (lane < 8 * HALVES) {   // 16-token pages: one 16-row box per page and half
+        const int pg = lane & 7, half = lane >> 3;
+        const int lp = c.tile * 8 + pg;
+        int page = 0;
+        if (lp * 16 < c.T) {
+          page = p.page_table[(size_t)c.b * p.max_pages + lp];
+          if (page < 0 || page >= p.n_pages) {
+            flag_status(ASP_DEV_BAD_PAGE);
+            page = 0;   // keeps the byte count; the rows' scores are not meaningful
+          }
+        }
+        tma_load_2d(sdst + half * (kTileT * 128) + pg * (16 * 128), &kmap, half * 64, (page * p.n_kv + c.h) * 16,
+                    &full[s], policy);
+      }
+      ++issued;
+      advance(c);
+    }
+    if (!done_ok) {   // a wait ran out: give the copies in flight a bounded chance to land
+      for (int k = max(0, issued - kStages); k < issued; ++k) mbar_wait(&full[k % kStages], (uint32_t)(k / kStages) & 1u);
+    }
+  } else if (n_my > 0 && warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    for (int k = 0; k < n_my; ++k) {
+      const int s = k % kStages;
+      const uint32_t ph = (uint32_t)(k / kStages) & 1u;
+      const int a = k & 1;
+      const uint32_t aph = (uint32_t)(k >> 1) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(&tempty[a], aph ^ 1u))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t st = sbase + s * STAGE;
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          const int half = kk / 4, k4 = kk % 4;
+          const uint64_t adesc = sw128_desc(st + half * (kTileT * 128) + k4 * 32);
+          const uint64_t bdesc = sw128_desc(st + KBYTES + half * (kN * 128) + k4 * 32);
+          umma_bf16(tmem + a * 16, adesc, bdesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+        umma_commit(&tfull[a]);
+      }
+      __syncwarp();
+    }
+  } else if (n_my > 0 && warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;   // TMEM lanes 32*quarter .. +31 belong to this warp
+    TileCursor c;
+    locate(t0, c);
+    for (int k = 0; k < n_my; ++k) {
+      const int a = k & 1;
+      const uint32_t aph = (uint32_t)(k >> 1) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[a], aph))) break;
+      tc_fence_after();
+      float v[16];
+      tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 16), v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[a]);
+      float m = v[0] + v[G];
+#pragma unroll
+      for (int g = 1; g < G; ++g) m = fmaxf(m, v[g] + v[G + g]);
+      const int j = c.tile * kTileT + quarter * 32 + lane;
+      const bool has = j < c.T;
+      if (has) p.scores[(size_t)(c.b * p.n_kv + c.h) * p.t_max + j] = m;
+      if (p.hist) {   // first radix pass of the selection, fused
+        const uint32_t dig = order_key(m) >> kTopShift;
+        const uint32_t hm = __ballot_sync(0xffffffffu, has);
+        if (has) {
+          const uint32_t peers = __match_any_sync(hm, dig);
+          if (lane == __ffs(peers) - 1)
+            atomicAdd(p.hist + (size_t)(c.b * p.n_kv + c.h) * kTopBins + dig, __popc(peers));
+        }
+      }
+      advance(c);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+template <int D, int G>
+cudaError_t launch_tc_t(const KvView& kv, const TcParams& p, cudaStream_t s) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t rows = kv.page_size ? (cuuint64_t)kv.n_pages * kv.n_kv * 16
+                                       : (cuuint64_t)kv.batch * kv.n_kv * kv.t_max;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, kv.page_size ? 16u : (cuuint32_t)kTileT};
+  const cuuint32_t estride[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kv.k), dims, strides, box, estride,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  constexpr int STAGE = kTileT * D * 2 + (D / 64) * kN * 128;
+  const size_t smem = 1024 + (size_t)kStages * STAGE + (2 * kStages + 4) * 8 + (2 * (size_t)p.batch + 1) * 4;
+  auto kern = score_tc_kernel<D, G>;
+  if (prepare_kernel((const void*)kern, smem, kThreadsTC) < 1) return cudaErrorInvalidConfiguration;
+  kern<<<sm_count(), kThreadsTC, smem, s>>>(map, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool score_tc_supported(const KvView& kv, int n_q_heads, const float* qpred) {
+  const int G = n_q_heads / kv.n_kv;
+  return !kv.kv_f32 && (kv.head_dim == 64 || kv.head_dim == 128) && (kv.page_size == 0 || kv.page_size == 16) &&
+         (G == 1 || G == 2 || G == 4 || G == 8) && kv.batch <= 8192 &&
+         (reinterpret_cast<uintptr_t>(qpred) & 15) == 0;
+}
+
+cudaError_t launch_score_tc(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s,
+                            int32_t* hist) {
+  TcParams p;
+  p.qpred = qpred;
+  p.n_q_heads = n_q_heads;
+  p.G = n_q_heads / kv.n_kv;
+  p.batch = kv.batch;
+  p.n_kv = kv.n_kv;
+  p.t_max = kv.t_max;
+  p.page_size = kv.page_size;
+  p.max_pages = kv.max_pages;
+  p.n_pages = kv.n_pages;
+  p.page_table = kv.page_table;
+  p.seq_lens = kv.seq_lens;
+  p.scores = scores;
+  p.hist = hist;
+  p.scale = 1.0f / sqrtf((float)kv.head_dim);
+  switch (p.G * (kv.head_dim == 64 ? 1 : -1)) {
+    case 1: return launch_tc_t<64, 1>(kv, p, s);
+    case 2: return launch_tc_t<64, 2>(kv, p, s);
+    case 4: return launch_tc_t<64, 4>(kv, p, s);
+    case 8: return launch_tc_t<64, 8>(kv, p, s);
+    case -1: return launch_tc_t<128, 1>(kv, p, s);
+    case -2: return launch_tc_t<128, 2>(kv, p, s);
+    case -4: return launch_tc_t<128, 4>(kv, p, s);
+    case -8: return launch_tc_t<128, 8>(kv, p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+ASP_STATUS_READER(read_status_score_tc)
+
+}  // namespace asp
