@@ -166,7 +166,7 @@ ASP_API asp_status asp_score_keys(const float* qpred, int n_q_heads, const asp_k
  * seq_lens : device int32 [batch] or NULL (T_b = t_max).
  * idx      : device int32 [batch, n_kv_heads, C], written.
  * count    : device int32 [batch, n_kv_heads], written.
- * Errors: ASP_ERR_INVALID_ARG; ASP_ERR_UNSUPPORTED (t_max > 262144). */
+ * Errors: ASP_ERR_INVALID_ARG; ASP_ERR_UNSUPPORTED (batch * n_kv_heads > 65535). */
 ASP_API asp_status asp_select_topk(const float* scores, const int32_t* seq_lens, int batch, int n_kv_heads,
                            int t_max, int C, int32_t* idx, int32_t* count, asp_stream_t stream);
 
@@ -244,6 +244,8 @@ ASP_API asp_status asp_sparse_attend_noalloc(const void* q, asp_dtype q_dtype, i
  *   s_side : waits for ev_fork (recorded on s_main at entry), pushes q_t into the
  *            ring, predicts qpred, scores every key, selects idx_next/count_next,
  *            then records ev_sel_done.
+ * The side chain is the step's critical path: s_side should be a stream of higher
+ * priority than s_main, so that its kernels get SMs before the attention's.
  * The caller swaps idx_cur/idx_next (and count_*) between steps, advances
  * ring_start by one, and must not reuse q_t, qpred, scores or idx_next before
  * ev_sel_done completes.  workspace: at least asp_decode_workspace_bytes(...)

@@ -263,7 +263,8 @@ class DecodeState:
         ws = int(lib().asp_decode_workspace_bytes(B, n_q_heads, Hkv, d, C, max_tail if tail_begin is not None else 0))
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
         self.s_main = s_main or torch.cuda.current_stream()
-        self.s_side = s_side or torch.cuda.Stream()
+        # the selection chain is the step's critical path: give it the highest priority
+        self.s_side = s_side or torch.cuda.Stream(priority=-100)
         self.ev_fork = make_event()
         self.ev_sel_done = make_event()
         self.timing_events = [make_event(True) for _ in range(8)] if timing else None
@@ -297,6 +298,15 @@ class DecodeState:
         a.ev_sel_done = event_handle(self.ev_sel_done)
         a.timing = ctypes.cast(self._timing_arr, POINTER(c_void_p)) if self._timing_arr is not None else None
         return a
+
+    def set_timing(self, on: bool) -> None:
+        """Record the per-kernel timing events in later steps (they sit between the
+        side stream's kernels, so they also keep those kernels from overlapping)."""
+        if on and self._timing_arr is None:
+            raise ValueError("DecodeState was created without timing events")
+        ptr = ctypes.cast(self._timing_arr, POINTER(c_void_p)) if on else None
+        for a in self._args:
+            a.timing = ptr
 
     def set_selection(self, idx: torch.Tensor, count: torch.Tensor) -> None:
         self.idx[self.cur].copy_(idx)

@@ -402,6 +402,7 @@ __global__ void __launch_bounds__(D) attend_merge_kernel(const float* __restrict
   using E = Elem<KT>;
   const size_t bh = blockIdx.x;
   const int c = threadIdx.x;
+  pdl_wait();   // the split partials come from the previous kernel
   const float* ml = part_ml + bh * splits * 2;
   float M = -INFINITY;
   for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[2 * s]);
@@ -432,8 +433,8 @@ cudaError_t launch_t(const AttParams& p, cudaStream_t s) {
   kern<<<dim3(p.splits, p.batch * p.n_kv), kWarps * 32, smem, s>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || p.splits == 1) return e;
-  attend_merge_kernel<KT, D><<<p.batch * p.n_q_heads, D, 0, s>>>(p.part_o, p.part_ml, p.splits, p.out, p.lse);
-  return cudaGetLastError();
+  return launch_pdl(attend_merge_kernel<KT, D>, dim3(p.batch * p.n_q_heads), dim3(D), 0, s, (const float*)p.part_o,
+                    (const float*)p.part_ml, p.splits, p.out, p.lse);
 }
 
 template <typename KT, int D>

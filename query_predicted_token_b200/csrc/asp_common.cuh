@@ -113,6 +113,14 @@ __device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32
       : "memory");
 }
 
+// ---- programmatic dependent launch --------------------------------------------
+// A kernel launched with programmatic stream serialisation may start while the
+// previous kernel of its stream is still running; pdl_wait() blocks until that
+// kernel has finished and its writes are visible (a no-op for normal launches).
+// pdl_trigger() lets the next kernel of the stream launch early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- selection keys ---------------------------------------------------------
 
 // 32-bit key whose unsigned order is the IEEE order of the score (-0.0 == +0.0).

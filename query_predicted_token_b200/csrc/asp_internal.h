@@ -5,6 +5,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 
 #include "asp.h"
@@ -18,6 +19,23 @@ int sm_count();
 // kernel's dynamic shared-memory limit and returns its resident CTAs per SM
 // (0 if the configuration cannot launch).  Cached, so launches stay cheap.
 int prepare_kernel(const void* kern, size_t smem, int threads);
+
+// Launches `kern` with programmatic stream serialisation: it may begin while the
+// previous kernel on `s` finishes (the kernel orders its reads with pdl_wait()).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Per-file device status readers (OR into *bits, then clear).
 cudaError_t read_status_predict(cudaStream_t s, int* bits);
@@ -84,6 +102,7 @@ struct SelectArgs {
   int32_t* idx;
   int32_t* count;
   const int32_t* hist0;      // optional first-pass histogram [n_rows, 2048] (expand == 1 only)
+  int key_cap;               // set by launch_select: keys kept in shared memory per row (0 = none)
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
 bool select_supported(int t_max, int expand);

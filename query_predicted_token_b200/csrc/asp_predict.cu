@@ -29,7 +29,7 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kLda = 33;   // row stride (doubles) of the lag Gram: column accesses hit distinct banks
-constexpr size_t kSolveBytes = (32 * kLda + 3 * 32) * 8;   // A[32][33], rhs, 1/diag, spare (fp64)
+constexpr size_t kSolveBytes = (32 * kLda + 3 * 32) * 8;   // A[32][33], rhs/beta, 1/diag, spare (fp64)
 
 template <int N, int OFF>
 struct ReduceScatterD {
@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head = blockIdx.x * kWarps + warp;
+  pdl_trigger();   // the key scan may launch and run its prologue meanwhile
   if (a.zero) {   // clear the next kernel's histogram (16-byte stores, spread over all warps)
     const size_t n4 = a.zero_words / 4;
     int4* z4 = reinterpret_cast<int4*>(a.zero);
@@ -160,26 +161,39 @@ __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
   __syncwarp();
 
   const int wm = a.wmax;
-  // Cholesky A = L L^T in place (lower triangle), right-looking.  Every lane
-  // computes the pivot; lane i owns row i; column k is broadcast by shuffles.
-  for (int k = 0; k < wm; ++k) {
-    const double dkk = sqrt(A[k * kLda + k]);
-    const double inv = 1.0 / dkk;
-    double lik = 0.0;
-    if (lane > k && lane < wm) {
-      lik = A[lane * kLda + k] * inv;
-      A[lane * kLda + k] = lik;
+  constexpr int WMAX = NV - 1;   // lags the registers can hold
+  // Cholesky A = L L^T with lane i holding row i of the lower triangle in
+  // registers; the pivot comes from lane k and column k is broadcast by shuffles.
+  {
+    double arow[WMAX];
+#pragma unroll
+    for (int j = 0; j < WMAX; ++j) arow[j] = (j <= lane && lane < wm && j < wm) ? A[lane * kLda + j] : 0.0;
+#pragma unroll
+    for (int k = 0; k < WMAX; ++k) {
+      if (k < wm) {
+        const double dkk = sqrt(__shfl_sync(0xffffffffu, arow[k], k));
+        const double inv = 1.0 / dkk;
+        const double lik = (lane > k && lane < wm) ? arow[k] * inv : 0.0;
+        if (lane == k) {
+          arow[k] = dkk;
+          invd[k] = inv;
+        } else if (lane > k) {
+          arow[k] = lik;
+        }
+#pragma unroll
+        for (int j = k + 1; j < WMAX; ++j) {
+          const double ljk = __shfl_sync(0xffffffffu, lik, j);
+          if (j < wm && lane >= j && lane < wm) arow[j] -= lik * ljk;
+        }
+      }
     }
-    if (lane == k) {
-      A[k * kLda + k] = dkk;
-      invd[k] = inv;
+    if (lane < wm) {
+#pragma unroll
+      for (int j = 0; j < WMAX; ++j)
+        if (j <= lane) A[lane * kLda + j] = arow[j];
     }
-    for (int j = k + 1; j < wm; ++j) {
-      const double ljk = __shfl_sync(0xffffffffu, lik, j);
-      if (lane >= j && lane < wm) A[lane * kLda + j] -= lik * ljk;
-    }
-    __syncwarp();
   }
+  __syncwarp();
   // forward substitution L z = rhs (shared by every window): lane i keeps z_i
   double z = lane < wm ? rhs[lane] : 0.0;
   for (int k = 0; k < wm; ++k) {
@@ -187,44 +201,79 @@ __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
     if (lane == k) z = zk;
     if (lane > k && lane < wm) z -= A[lane * kLda + k] * zk;
   }
-
+  // Back substitutions L_w^T a = z_w for all windows at once: window wi owns the
+  // lanes [base_wi, base_wi + w) (in rounds if the widths exceed 32).  The
+  // weights are folded into beta_r = sum_w alpha_{w,r}, so that
+  // qhat = (1/|windows|) sum_r beta_r q_{t-r}.
+  double* beta = rhs;   // rhs is no longer needed: reuse it for beta
+  if (lane < 32) beta[lane] = 0.0;
+  __syncwarp();
+  int win[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) win[k] = a.windows[k];
+  for (int first = 0; first < a.n_win;) {
+    int last = first, used = 0;   // windows [first, last) share this round
+    while (last < a.n_win && used + win[last] <= 32) used += win[last++];
+    int my_w = 0, my_base = 0, base = 0;
+    for (int k = first; k < last; ++k) {
+      if (lane >= base && lane < base + win[k]) {
+        my_w = win[k];
+        my_base = base;
+      }
+      base += win[k];
+    }
+    const int li = lane - my_base;   // this lane's lag index in its window
+    double av = (my_w > 0) ? __shfl_sync(0xffffffffu, z, li) : __shfl_sync(0xffffffffu, z, 0);
+    int kmax = 0;
+    for (int k = first; k < last; ++k) kmax = max(kmax, win[k]);
+    for (int k = kmax - 1; k >= 0; --k) {
+      const bool act = k < my_w;
+      const double ak = __shfl_sync(0xffffffffu, av, act ? my_base + k : lane) * invd[k];
+      if (act && li == k) av = ak;
+      if (act && li < k) av -= A[k * kLda + li] * ak;
+    }
+    // weights over each window's lags (softmax within the window unless raw)
+    double wgt = av;
+    if (!a.coef_raw) {   // one exp per lane; maxima and sums over the window through shared memory
+      double* tmp = invd + 32;   // 32 spare doubles
+      tmp[lane] = (my_w > 0) ? av : 0.0;
+      __syncwarp();
+      double m = -INFINITY;
+      for (int r = 0; r < my_w; ++r) m = fmax(m, tmp[my_base + r]);
+      const double e = (my_w > 0) ? exp(av - m) : 0.0;
+      __syncwarp();
+      tmp[lane] = e;
+      __syncwarp();
+      double zs = 0.0;
+      for (int r = 0; r < my_w; ++r) zs += tmp[my_base + r];
+      wgt = (my_w > 0) ? e / zs : 0.0;
+      __syncwarp();
+    }
+    // beta_r += weight of lag r in each window of the round
+    double* tmp2 = invd + 32;
+    tmp2[lane] = (my_w > 0) ? wgt : 0.0;
+    __syncwarp();
+    if (lane < WMAX) {
+      double add = 0.0;
+      int bb = 0;
+      for (int k = first; k < last; ++k) {
+        if (lane < win[k]) add += tmp2[bb + lane];
+        bb += win[k];
+      }
+      beta[lane] += add;
+    }
+    __syncwarp();
+    first = last;
+  }
   float acc[CPL];
 #pragma unroll
   for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
-  for (int wi = 0; wi < a.n_win; ++wi) {
-    int w = 0;   // a.windows[wi] without a dynamically indexed copy of the parameters
+  const float bl = lane < WMAX ? (float)beta[lane] : 0.f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-      if (k == wi) w = a.windows[k];
-    // back substitution L_w^T a = z_w on the leading w x w block: lane i keeps a_i
-    double av = lane < w ? z : 0.0;
-    for (int k = w - 1; k >= 0; --k) {
-      const double ak = __shfl_sync(0xffffffffu, av, k) * invd[k];
-      if (lane == k) av = ak;
-      if (lane < k) av -= A[k * kLda + lane] * ak;
-    }
-    // weights over the w lags
-    double wgt = lane < w ? av : 0.0;
-    if (!a.coef_raw) {
-      double m = lane < w ? wgt : -INFINITY;
+  for (int r = 0; r < NV - 1; ++r) {   // lag r (q_{t-1-r}) weights q_{t-r} = h[r]
+    const float br = __shfl_sync(0xffffffffu, bl, r);
 #pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
-      const double e = lane < w ? exp(wgt - m) : 0.0;
-      double zs = e;
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
-      wgt = e / zs;
-    }
-    // lag r (q_{t-1-r}) weights the vector one step later, q_{t-r} = h[r]
-    const float wf = (float)wgt;
-#pragma unroll
-    for (int r = 0; r < NV - 1; ++r) {
-      const float wr = __shfl_sync(0xffffffffu, wf, r);
-      if (r < w) {
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) acc[c] = fmaf(wr, h[r][c], acc[c]);
-      }
-    }
+    for (int c = 0; c < CPL; ++c) acc[c] = fmaf(br, h[r][c], acc[c]);
   }
   float* out = a.qpred + (size_t)head * D + lane * CPL;
   const float inv_nw = 1.f / (float)a.n_win;

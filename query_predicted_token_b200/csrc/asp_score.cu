@@ -63,6 +63,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) score_kernel(ScoreParams p) {
   int* pre = reinterpret_cast<int*>(smem + (size_t)WARPS * STAGES * BLOCK_BYTES + WARPS * STAGES * 8);
   int* lens = pre + p.batch + 1;
 
+  pdl_wait();      // inputs may come from the previous kernel (the predicted queries, the cleared histogram)
+  pdl_trigger();
   for (int b = threadIdx.x; b < p.batch; b += blockDim.x) {
     int t = p.seq_lens ? p.seq_lens[b] : p.t_max;
     lens[b] = t < 0 ? 0 : (t > p.t_max ? p.t_max : t);
@@ -258,8 +260,7 @@ cudaError_t launch_score_t(const ScoreParams& p, cudaStream_t s) {
   const size_t smem = (size_t)WARPS * STAGES * BLOCK_BYTES + WARPS * STAGES * 8 + (2 * (size_t)p.batch + 1) * 4;
   const int per_sm = prepare_kernel((const void*)kern, smem, WARPS * 32);
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  kern<<<sm_count() * per_sm, WARPS * 32, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(sm_count() * per_sm), dim3(WARPS * 32), smem, s, p);
 }
 
 template <typename KT, int D>

@@ -129,12 +129,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_co
   int* lens = pre + p.batch + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  for (int b = threadIdx.x; b < p.batch; b += blockDim.x) {
-    int t = p.seq_lens ? p.seq_lens[b] : p.t_max;
-    lens[b] = t < 0 ? 0 : (t > p.t_max ? p.t_max : t);
-  }
-  __syncthreads();
-  cta_prefix_sum(p.batch, pre, [&](int b) { return ((lens[b] + kTileT - 1) / kTileT) * p.n_kv; }, scratch);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -151,6 +145,17 @@ __global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_co
                  "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
+  // Everything above touches no global memory, so it overlaps the previous
+  // kernel; the predicted queries, the cleared histogram and the cache
+  // description are read only after it has finished.
+  pdl_wait();
+  pdl_trigger();   // the selection may launch while the scan runs
+  for (int b = threadIdx.x; b < p.batch; b += blockDim.x) {
+    int t = p.seq_lens ? p.seq_lens[b] : p.t_max;
+    lens[b] = t < 0 ? 0 : (t > p.t_max ? p.t_max : t);
+  }
+  __syncthreads();
+  cta_prefix_sum(p.batch, pre, [&](int b) { return ((lens[b] + kTileT - 1) / kTileT) * p.n_kv; }, scratch);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -196,6 +201,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_co
     locate(t0, c);
     int qb = -1, qh = -1;
     uint4 qreg[QCH];
+    int pt_b = -1, pt_base = 0, pt_val = -1, pt_next = -1;
     int issued = 0, done_ok = 1;
     for (int k = 0; k < n_my; ++k) {
       const int s = k % kStages;
@@ -248,19 +254,35 @@ __global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_co
           const int y = (c.b * p.n_kv + c.h) * p.t_max + c.tile * kTileT;
           tma_load_2d(sdst + lane * (kTileT * 128), &kmap, lane * 64, y, &full[s], policy);
         }
-      } else if (lane < 8 * HALVES) {   // 16-token pages: one 16-row box per page and half
+      } else {   // 16-token pages: one 16-row box per page and half
+        // page-table window: lane l holds entry pt_base + l of row pt_b; the next
+        // window is loaded one window ahead, so table lookups stay off the
+        // critical path
+        const int lp0 = c.tile * 8;
+        if (c.b != pt_b || lp0 < pt_base || lp0 + 8 > pt_base + 32) {
+          if (c.b == pt_b && lp0 == pt_base + 32) {
+            pt_val = pt_next;
+          } else {
+            const int e = lp0 + lane;
+            pt_val = e < p.max_pages ? p.page_table[(size_t)c.b * p.max_pages + e] : -1;
+          }
+          pt_b = c.b;
+          pt_base = lp0;
+          const int e = lp0 + 32 + lane;
+          pt_next = e < p.max_pages ? p.page_table[(size_t)c.b * p.max_pages + e] : -1;
+        }
         const int pg = lane & 7, half = lane >> 3;
-        const int lp = c.tile * 8 + pg;
-        int page = 0;
-        if (lp * 16 < c.T) {
-          page = p.page_table[(size_t)c.b * p.max_pages + lp];
-          if (page < 0 || page >= p.n_pages) {
+        int page = __shfl_sync(0xffffffffu, pt_val, lp0 - pt_base + pg);
+        if (lane < 8 * HALVES) {
+          if ((lp0 + pg) * 16 >= c.T) {
+            page = 0;   // past the sequence: any valid page keeps the byte count
+          } else if (page < 0 || page >= p.n_pages) {
             flag_status(ASP_DEV_BAD_PAGE);
             page = 0;   // keeps the byte count; the rows' scores are not meaningful
           }
+          tma_load_2d(sdst + half * (kTileT * 128) + pg * (16 * 128), &kmap, half * 64,
+                      (page * p.n_kv + c.h) * 16, &full[s], policy);
         }
-        tma_load_2d(sdst + half * (kTileT * 128) + pg * (16 * 128), &kmap, half * 64, (page * p.n_kv + c.h) * 16,
-                    &full[s], policy);
       }
       ++issued;
       advance(c);
@@ -368,8 +390,7 @@ cudaError_t launch_tc_t(const KvView& kv, const TcParams& p, cudaStream_t s) {
   const size_t smem = 1024 + (size_t)kStages * STAGE + (2 * kStages + 4) * 8 + (2 * (size_t)p.batch + 1) * 4;
   auto kern = score_tc_kernel<D, G>;
   if (prepare_kernel((const void*)kern, smem, kThreadsTC) < 1) return cudaErrorInvalidConfiguration;
-  kern<<<sm_count(), kThreadsTC, smem, s>>>(map, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(sm_count()), dim3(kThreadsTC), smem, s, map, p);
 }
 
 }  // namespace

@@ -118,7 +118,6 @@ def test_score_rejects_bad_groups(lib):
 def test_select_validation(lib):
     assert lib.asp_select_topk(FAKE, None, 2, 2, 1024, 0, FAKE, FAKE, None) == L.ASP_ERR_INVALID_ARG
     assert lib.asp_select_topk(None, None, 2, 2, 1024, 8, FAKE, FAKE, None) == L.ASP_ERR_INVALID_ARG
-    assert lib.asp_select_topk(FAKE, None, 2, 2, 300000, 8, FAKE, FAKE, None) == L.ASP_ERR_UNSUPPORTED
     assert lib.asp_select_topk(FAKE, None, 70000, 1, 1024, 8, FAKE, FAKE, None) == L.ASP_ERR_UNSUPPORTED
 
 
