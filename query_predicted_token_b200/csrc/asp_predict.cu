@@ -31,27 +31,13 @@ constexpr int kWarps = 4;
 constexpr int kLda = 33;   // row stride (doubles) of the lag Gram: column accesses hit distinct banks
 constexpr size_t kSolveBytes = (32 * kLda + 3 * 32) * 8;   // A[32][33], rhs/beta, 1/diag, spare (fp64)
 
-template <int N, int OFF>
-struct ReduceScatterD {
-  __device__ __forceinline__ static void run(double* vals, int lane) {
-    if constexpr (OFF >= 1) {
-      if constexpr (N >= 2) {
-        constexpr int H = N / 2;
-        const bool upper = (lane & OFF) != 0;
-#pragma unroll
-        for (int i = 0; i < H; ++i) {
-          const double send = upper ? vals[i] : vals[i + H];
-          const double keep = upper ? vals[i + H] : vals[i];
-          vals[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
-        }
-        ReduceScatterD<H, OFF / 2>::run(vals, lane);
-      } else {
-        vals[0] += __shfl_xor_sync(0xffffffffu, vals[0], OFF);
-        ReduceScatterD<1, OFF / 2>::run(vals, lane);
-      }
-    }
-  }
-};
+// 1/sqrt(x) for x > 0 in fp64: the fp32 hardware estimate refined by one
+// Newton-Raphson step y <- y (3 - x y^2) / 2, which squares its relative error
+// (about 1e-7 -> 1e-14) at the cost of four fp64 operations.
+__device__ __forceinline__ double rsqrt_f64(double x) {
+  const double y = (double)rsqrtf((float)x);
+  return y * (1.5 - 0.5 * x * y * y);
+}
 
 // Stores the reduced pair `q` (lane's pair of a round) into the solve arrays:
 // pairs (i >= 1, j >= 1) are lag-Gram entries, pairs (i >= 1, 0) the right-hand side.
@@ -171,8 +157,9 @@ __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
 #pragma unroll
     for (int k = 0; k < WMAX; ++k) {
       if (k < wm) {
-        const double dkk = sqrt(__shfl_sync(0xffffffffu, arow[k], k));
-        const double inv = 1.0 / dkk;
+        const double akk = __shfl_sync(0xffffffffu, arow[k], k);
+        const double inv = rsqrt_f64(akk);   // 1 / L_kk
+        const double dkk = akk * inv;        // L_kk = sqrt(A_kk)
         const double lik = (lane > k && lane < wm) ? arow[k] * inv : 0.0;
         if (lane == k) {
           arow[k] = dkk;
@@ -240,7 +227,7 @@ __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
       __syncwarp();
       double m = -INFINITY;
       for (int r = 0; r < my_w; ++r) m = fmax(m, tmp[my_base + r]);
-      const double e = (my_w > 0) ? exp(av - m) : 0.0;
+      const double e = (my_w > 0) ? (double)expf((float)(av - m)) : 0.0;
       __syncwarp();
       tmp[lane] = e;
       __syncwarp();
