@@ -345,7 +345,7 @@ def main():
     peak, peak_kind = read_peaks()
     score_ms = statistics.mean(kern_ms["score"])
     achieved = acct["score"] / (score_ms / 1e3) / 1e9
-    traffic = read_traffic("asp_score.cu", 1.0) if wl.name == "qwen3_8b_shaped_32k" else None
+    traffic = read_traffic("asp_score_tc.cu", 1.0) if wl.name == "qwen3_8b_shaped_32k" else None
 
     if rank == 0:
         cpu = None
@@ -367,7 +367,7 @@ def main():
             "step_us_p90": round(sorted(step_ms)[int(0.9 * (len(step_ms) - 1))] * 1e3, 2),
             "kernel_us": {n: round(statistics.mean(v) * 1e3, 2) for n, v in kern_ms.items()},
             "step_bytes": acct["total"],
-            "roofline": {"kernel": "score_keys", "bound": "hbm", "achieved": round(achieved, 1),
+            "roofline": {"kernel": "score_tc_kernel (key scan)", "bound": "hbm", "achieved": round(achieved, 1),
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": traffic, "algorithmic_bytes": acct["score"]},
             "step_frac_of_peak": round(value / world / peak, 4),
