@@ -244,21 +244,19 @@ def main():
     if args.impl == "reference":
         return run_reference(args)
     import torch
-    import torch.distributed as dist
     import query_predicted_token_b200 as asp
     import synth
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+    from query_predicted_token_b200.replicas import ReplicaGroup, rank_workload
+
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    group = ReplicaGroup("nccl", dev, timeout_s=120)
+    world, rank = group.world, group.rank
 
     asp.lib()   # raises if the library is missing: there is no other path
-    wl = synth.workload(args.workload)
+    wl = rank_workload(synth.workload(args.workload), rank)   # each rank: its own batch
     B, Hq, Hkv, d, C = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.C
     kvd = synth.kv_cache(wl, dev)
     lens = kvd["seq_lens"].cpu().tolist()
@@ -300,8 +298,7 @@ def main():
     for _ in range(max(3, args.warmup)):
         one_step()
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    group.barrier()
     gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
     gpu_id = gpu_id if gpu_id.startswith("GPU-") else "GPU-" + gpu_id
     kern_ms = {n: [] for n in ("predict", "score", "select", "attend")}
@@ -332,14 +329,9 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = [a.elapsed_time(b) for a, b in ev]
 
-    t_rank = sum(step_ms) / 1e3
-    t_e2e = sum(e2e_ms) / 1e3
-    if world > 1:
-        t = torch.tensor([t_rank, t_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_rank, t_e2e = t.tolist()
-        dist.barrier()
-    total_bytes = acct["total"] * args.steps * world
+    t_rank, t_e2e = group.slowest(sum(step_ms) / 1e3, sum(e2e_ms) / 1e3)
+    (total_bytes,) = group.total(acct["total"] * args.steps)   # ragged batches differ per rank
+    group.barrier()
     value = total_bytes / t_rank / 1e9
     e2e_value = total_bytes / t_e2e / 1e9
     peak, peak_kind = read_peaks()
@@ -378,9 +370,7 @@ def main():
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    group.close()
     return 0
 
 
