@@ -394,6 +394,308 @@ __global__ void __launch_bounds__(kWarps * 32) attend_kernel(AttParams p) {
   }
 }
 
+// ---- bf16 cache with a bf16 query: both small contractions on tensor cores ----
+//
+// Per 16-row tile a warp computes S^T[head x row] = Q[head x d] . K^T with
+// mma.m16n8k16 (M = query heads, G <= 8 of the 16 rows used; N = 8 rows per
+// n-tile; K = 16 channels), takes the online softmax in fp32, splits the
+// probabilities into bf16 hi and lo parts and accumulates O[head x d] +=
+// P[head x row] . V with two more mmas (K = the 16 rows); the accumulator
+// layout of the logits is the operand layout of P.  The query and the cache are
+// bf16, so every product is exact and only fp32 summation order differs from a
+// CUDA-core dot product.  K and V rows sit in shared memory at a 16-byte padded
+// stride, so the eight rows an ldmatrix phase reads fall in distinct banks.
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// d01 += A . B on the top 8 rows of a 16x8 tile; the A rows 8-15 are zero, so
+// their accumulators are not kept.  a0: (row g, k 2t..2t+1), a2: (row g, k
+// 8+2t..9+2t); b0: (k 2t..2t+1, col g), b1: (k 8+2t..9+2t, col g).
+__device__ __forceinline__ void mma_top8(float& d0, float& d1, uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  float x2, x3;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %11, %12, %13};"
+      : "=f"(d0), "=f"(d1), "=f"(x2), "=f"(x3)
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d0), "f"(d1), "f"(0.f), "f"(0.f));
+}
+
+// (x0, x1) -> hi = bf16 pair rn(x), lo = bf16 pair rn(x - hi); x0 in the low half.
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+template <int D, int G, int STAGES>
+__global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
+  constexpr int ROW_BYTES = D * 2;
+  constexpr int STRIDE = ROW_BYTES + 16;          // padded row pitch in shared memory
+  constexpr int HALF = kTile * STRIDE;            // the K (or V) rows of one stage
+  constexpr int TILE_BYTES = 2 * HALF;
+  constexpr int KS = D / 16;                      // k-steps of the logits
+  constexpr int NT = D / 8;                       // n-tiles of the output
+  static_assert(G >= 1 && G <= 8 && kTile == 16, "layout");
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;          // fragment row (query head) and column pair
+  uint8_t* wbuf = smem + (size_t)warp * STAGES * TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kWarps * STAGES * TILE_BYTES) + warp * STAGES;
+
+  const int unit = blockIdx.y, split = blockIdx.x;
+  const int b = unit / p.n_kv, h = unit - b * p.n_kv;
+  int T = p.seq_lens ? p.seq_lens[b] : p.t_max;
+  T = T < 0 ? 0 : (T > p.t_max ? p.t_max : T);
+  int n_sel = (p.C > 0 && p.count) ? p.count[unit] : 0;
+  n_sel = n_sel < 0 ? 0 : (n_sel > p.C ? p.C : n_sel);
+  int tb = T;
+  if (p.tail_begin) {
+    tb = p.tail_begin[b];
+    tb = tb < 0 ? 0 : (tb > T ? T : tb);
+  }
+  int tail = T - tb;
+  if (tail > p.max_tail) {
+    if (threadIdx.x == 0 && split == 0) flag_status(ASP_DEV_TAIL_LIMIT);
+    tail = p.max_tail;
+  }
+  const int n_rows = n_sel + tail;
+  const int r0 = split * p.rows_per_split;
+  const int r1 = min(n_rows, r0 + p.rows_per_split);
+  const int n_tiles = r1 > r0 ? (r1 - r0 + kTile - 1) / kTile : 0;
+  const int32_t* idx_row = n_sel ? p.idx + (size_t)unit * p.C : nullptr;
+
+  if (lane == 0) {
+    for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+
+  // query fragments: head g (zero rows for g >= G), channels 16kk + 2t (+8)
+  uint32_t qa[KS][2];
+  {
+    const __nv_bfloat16* qrow =
+        static_cast<const __nv_bfloat16*>(p.q) + (size_t)(b * p.n_q_heads + h * G + (g < G ? g : 0)) * D;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      qa[kk][0] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t) : 0u;
+      qa[kk][1] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 8 + 2 * t) : 0u;
+    }
+  }
+
+  const int my_tiles = n_tiles > warp ? (n_tiles - warp + kWarps - 1) / kWarps : 0;
+
+  struct RowSrc {
+    const uint8_t* src;
+    bool valid;
+  };
+  // Row source of this lane for tile t (lanes 0-15: K rows, 16-31: V rows).
+  auto resolve = [&](int tt) -> RowSrc {
+    const int rr = lane & 15;
+    const bool isv = lane >= 16;
+    const int r = r0 + (warp + tt * kWarps) * kTile + rr;
+    bool valid = r < r1;
+    int j = 0;
+    if (valid) {
+      if (r < n_sel) {
+        j = idx_row[r];
+        if (j < 0 || j >= T) {
+          valid = false;
+          if (!isv) flag_status(ASP_DEV_BAD_INDEX);
+        } else if (j >= tb) {
+          valid = false;   // covered by the tail
+        }
+      } else {
+        j = tb + (r - n_sel);
+      }
+    }
+    const uint8_t* src = nullptr;
+    if (valid) {
+      const uint8_t* base = isv ? p.v : p.k;
+      if (p.page_size == 0) {
+        src = base + ((size_t)unit * p.t_max + j) * ROW_BYTES;
+      } else {
+        const int page = p.page_table[(size_t)b * p.max_pages + j / p.page_size];
+        if (page < 0 || page >= p.n_pages) {
+          valid = false;
+          if (!isv) flag_status(ASP_DEV_BAD_PAGE);
+        } else {
+          src = base + (((size_t)page * p.n_kv + h) * p.page_size + (j % p.page_size)) * ROW_BYTES;
+        }
+      }
+    }
+    return RowSrc{src, valid};
+  };
+  auto issue = [&](const RowSrc& rs, int slot) -> uint32_t {
+    const int rr = lane & 15;
+    const bool isv = lane >= 16;
+    const uint32_t vm = __ballot_sync(0xffffffffu, rs.valid) & 0xffffu;
+    uint8_t* dst = wbuf + slot * TILE_BYTES + (isv ? HALF : 0) + rr * STRIDE;
+    if (!rs.valid) {
+#pragma unroll
+      for (int c = 0; c < ROW_BYTES / 16; ++c) reinterpret_cast<uint4*>(dst)[c] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)__popc(vm) * 2u * ROW_BYTES);
+    __syncwarp();
+    if (rs.valid) bulk_g2s(dst, rs.src, ROW_BYTES, &bars[slot]);
+    return vm;
+  };
+
+  float o[NT][2];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = 0.f;
+  float m_run = -INFINITY;   // running max (base 2) of head g
+  float l_run = 0.f;         // this lane's share of head g's running sum
+
+  // ldmatrix row addresses (byte offsets in a stage): lane l feeds row l & 7 of
+  // matrix l >> 3
+  const int mat = lane >> 3, mrow = lane & 7;
+  const uint32_t k_off = (uint32_t)(((mat >> 1) * 8 + mrow) * STRIDE + (mat & 1) * 16);        // + 32 kk
+  const uint32_t v_off = (uint32_t)(HALF + ((mat & 1) * 8 + mrow) * STRIDE + (mat >> 1) * 16);  // + 32 j
+
+  uint32_t vmask[STAGES];
+  int issued = 0;
+#pragma unroll 1
+  for (int s = 0; s < STAGES && s < my_tiles; ++s) {
+    vmask[s] = issue(resolve(s), s);
+    ++issued;
+  }
+  RowSrc next = issued < my_tiles ? resolve(issued) : RowSrc{nullptr, false};
+
+  int consumed = 0;
+  bool ok = true;
+#pragma unroll 1
+  for (int tt = 0; tt < my_tiles; ++tt) {
+    const int slot = tt % STAGES;
+    ok = __all_sync(0xffffffffu, mbar_wait(&bars[slot], (uint32_t)(tt / STAGES) & 1u));
+    if (!ok) break;
+    ++consumed;
+    const uint32_t vm = vmask[slot];
+    const uint32_t base = smem_u32(wbuf + slot * TILE_BYTES);
+
+    // 1. logits: n-tile 0 = rows 0-7, n-tile 1 = rows 8-15
+    float s0[2] = {0.f, 0.f}, s1[2] = {0.f, 0.f};
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      uint32_t kb[4];
+      ldsm_x4(kb, base + k_off + 32 * kk);
+      mma_top8(s0[0], s0[1], qa[kk][0], qa[kk][1], kb[0], kb[1]);
+      mma_top8(s1[0], s1[1], qa[kk][0], qa[kk][1], kb[2], kb[3]);
+    }
+
+    // 2. online softmax of head g over its 16 rows (4 per lane, 4 lanes per head)
+    float x[4] = {s0[0] * p.qscale, s0[1] * p.qscale, s1[0] * p.qscale, s1[1] * p.qscale};
+    const int rows[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
+    float mloc = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (!((vm >> rows[e]) & 1u)) x[e] = -INFINITY;
+      mloc = fmaxf(mloc, x[e]);
+    }
+    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+    const float m_new = fmaxf(m_run, mloc);
+    const float corr = (m_new == -INFINITY) ? 1.f : ex2(m_run - m_new);
+    float pr[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) pr[e] = (x[e] == -INFINITY) ? 0.f : ex2(x[e] - m_new);
+    l_run = l_run * corr + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
+    m_run = m_new;
+    // P as bf16 hi + lo parts: the products with bf16 V are exact in fp32, so
+    // the weights keep ~16 significant bits
+    uint32_t pa0, pa2, pl0, pl2;
+    split_bf16x2(pr[0], pr[1], pa0, pl0);
+    split_bf16x2(pr[2], pr[3], pa2, pl2);
+
+    // 3. O = O * corr + P . V
+    if (corr != 1.f) {
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        o[n][0] *= corr;
+        o[n][1] *= corr;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < D / 16; ++j) {
+      uint32_t vb[4];
+      ldsm_x4_trans(vb, base + v_off + 32 * j);
+      mma_top8(o[2 * j][0], o[2 * j][1], pa0, pa2, vb[0], vb[1]);
+      mma_top8(o[2 * j + 1][0], o[2 * j + 1][1], pa0, pa2, vb[2], vb[3]);
+      mma_top8(o[2 * j][0], o[2 * j][1], pl0, pl2, vb[0], vb[1]);
+      mma_top8(o[2 * j + 1][0], o[2 * j + 1][1], pl0, pl2, vb[2], vb[3]);
+    }
+    __syncwarp();
+    if (issued < my_tiles) {
+      vmask[slot] = issue(next, slot);
+      ++issued;
+      if (issued < my_tiles) next = resolve(issued);
+    }
+  }
+  if (!ok) {
+    for (int k = consumed + 1; k < issued; ++k) mbar_wait(&bars[k % STAGES], (uint32_t)(k / STAGES) & 1u);
+  }
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+
+  // combine the warps (shared memory reused from the stages)
+  __syncthreads();
+  float* mo = reinterpret_cast<float*>(smem);   // [kWarps][G][D] outputs, then [kWarps][G][2] (m, l)
+  float* mml = mo + kWarps * G * D;
+  if (g < G) {
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+      *reinterpret_cast<float2*>(mo + (warp * G + g) * D + n * 8 + 2 * t) = make_float2(o[n][0], o[n][1]);
+    if (t == 0) {
+      mml[(warp * G + g) * 2 + 0] = m_run;
+      mml[(warp * G + g) * 2 + 1] = l_run;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < G * D; e += kWarps * 32) {
+    const int gg = e / D, c = e - gg * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mml[(w * G + gg) * 2]);
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float mw = mml[(w * G + gg) * 2];
+        if (mw == -INFINITY) continue;
+        const float f = ex2(mw - M);
+        L += mml[(w * G + gg) * 2 + 1] * f;
+        O += mo[(w * G + gg) * D + c] * f;
+      }
+    }
+    const size_t bh = (size_t)b * p.n_q_heads + h * G + gg;
+    if (p.splits == 1) {
+      const float r = L > 0.f ? O / L : 0.f;
+      static_cast<__nv_bfloat16*>(p.out)[bh * D + c] = __float2bfloat16_rn(r);
+      if (c == 0 && p.lse) p.lse[bh] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+    } else {
+      p.part_o[(bh * p.splits + split) * D + c] = O;
+      if (c == 0) {
+        p.part_ml[(bh * p.splits + split) * 2 + 0] = M;
+        p.part_ml[(bh * p.splits + split) * 2 + 1] = L;
+      }
+    }
+  }
+}
+
 // Log-sum-exp merge of the split partials: one CTA of D threads per query head.
 template <typename KT, int D>
 __global__ void __launch_bounds__(D) attend_merge_kernel(const float* __restrict__ part_o,
@@ -435,6 +737,33 @@ cudaError_t launch_t(const AttParams& p, cudaStream_t s) {
   if (e != cudaSuccess || p.splits == 1) return e;
   return launch_pdl(attend_merge_kernel<KT, D>, dim3(p.batch * p.n_q_heads), dim3(D), 0, s, (const float*)p.part_o,
                     (const float*)p.part_ml, p.splits, p.out, p.lse);
+}
+
+template <int D, int G>
+cudaError_t launch_mma(const AttParams& p, cudaStream_t s) {
+  constexpr int STAGES = 2;
+  constexpr int TILE_BYTES = 2 * kTile * (D * 2 + 16);
+  auto kern = attend_mma_kernel<D, G, STAGES>;
+  size_t smem = (size_t)kWarps * STAGES * TILE_BYTES + kWarps * STAGES * 8;
+  const size_t merge = (size_t)kWarps * G * (D + 2) * 4;
+  if (smem < merge) smem = merge;
+  if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
+  kern<<<dim3(p.splits, p.batch * p.n_kv), kWarps * 32, smem, s>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || p.splits == 1) return e;
+  return launch_pdl(attend_merge_kernel<__nv_bfloat16, D>, dim3(p.batch * p.n_q_heads), dim3(D), 0, s,
+                    (const float*)p.part_o, (const float*)p.part_ml, p.splits, p.out, p.lse);
+}
+
+template <int D>
+cudaError_t dispatch_mma(int G, const AttParams& p, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_mma<D, 1>(p, s);
+    case 2: return launch_mma<D, 2>(p, s);
+    case 4: return launch_mma<D, 4>(p, s);
+    case 8: return launch_mma<D, 8>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 template <typename KT, int D>
@@ -513,6 +842,7 @@ cudaError_t launch_attend(const void* q, int q_f32, int n_q_heads, const KvView&
   p.qscale = kLog2e / sqrtf((float)kv.head_dim);
   const int G = n_q_heads / kv.n_kv;
   if (kv.kv_f32) return kv.head_dim == 64 ? dispatch_g<float, 64>(G, p, s) : dispatch_g<float, 128>(G, p, s);
+  if (!q_f32) return kv.head_dim == 64 ? dispatch_mma<64>(G, p, s) : dispatch_mma<128>(G, p, s);
   return kv.head_dim == 64 ? dispatch_g<__nv_bfloat16, 64>(G, p, s) : dispatch_g<__nv_bfloat16, 128>(G, p, s);
 }
 

@@ -62,6 +62,7 @@ struct PredictArgs {
   double lam;
   int coef_raw;
   float* qpred;
+  int win_fast;           // set by launch_predict: windows sorted, powers of two, one round of lanes
 };
 cudaError_t launch_predict(const PredictArgs& a, cudaStream_t s);
 

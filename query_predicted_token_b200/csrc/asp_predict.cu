@@ -86,7 +86,7 @@ struct GramRows {
 };
 
 template <int D, int NV>
-__global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, 1) predict_kernel(PredictArgs a) {
   constexpr int CPL = D / 32;   // contiguous channels per lane
   extern __shared__ __align__(16) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -198,6 +198,7 @@ __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
   int win[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) win[k] = a.windows[k];
+  float bfast = 0.f;   // beta of lag `lane` on the fast path
   for (int first = 0; first < a.n_win;) {
     int last = first, used = 0;   // windows [first, last) share this round
     while (last < a.n_win && used + win[last] <= 32) used += win[last++];
@@ -218,6 +219,35 @@ __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
       const double ak = __shfl_sync(0xffffffffu, av, act ? my_base + k : lane) * invd[k];
       if (act && li == k) av = ak;
       if (act && li < k) av -= A[k * kLda + li] * ak;
+    }
+    if (a.win_fast) {
+      // Windows of 2^j lanes at multiples of their width: maxima and sums over a
+      // window are xor butterflies, and lag r gathers its weights by shuffles.
+      float w32 = my_w > 0 ? (float)av : 0.f;
+      if (!a.coef_raw) {
+        float m = my_w > 0 ? w32 : -INFINITY;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float y = __shfl_xor_sync(0xffffffffu, m, o);
+          if (o < my_w) m = fmaxf(m, y);
+        }
+        const float ex = my_w > 0 ? expf(w32 - m) : 0.f;
+        float zs = ex;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float y = __shfl_xor_sync(0xffffffffu, zs, o);
+          if (o < my_w) zs += y;
+        }
+        w32 = my_w > 0 ? ex / zs : 0.f;
+      }
+      int bb = 0;
+      for (int k = first; k < last; ++k) {
+        const float v = __shfl_sync(0xffffffffu, w32, bb + (lane < win[k] ? lane : 0));
+        if (lane < win[k]) bfast += v;
+        bb += win[k];
+      }
+      first = last;
+      continue;
     }
     // weights over each window's lags (softmax within the window unless raw)
     double wgt = av;
@@ -255,7 +285,7 @@ __global__ void __launch_bounds__(kWarps * 32) predict_kernel(PredictArgs a) {
   float acc[CPL];
 #pragma unroll
   for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
-  const float bl = lane < WMAX ? (float)beta[lane] : 0.f;
+  const float bl = lane < WMAX ? (a.win_fast ? bfast : (float)beta[lane]) : 0.f;
 #pragma unroll
   for (int r = 0; r < NV - 1; ++r) {   // lag r (q_{t-1-r}) weights q_{t-r} = h[r]
     const float br = __shfl_sync(0xffffffffu, bl, r);
@@ -288,7 +318,24 @@ cudaError_t launch_d(const PredictArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_predict(const PredictArgs& a, cudaStream_t s) {
+cudaError_t launch_predict(const PredictArgs& args, cudaStream_t s) {
+  // The mean over the windows does not depend on their order: sort them widest
+  // first, so that windows whose widths are powers of two and add up to at most
+  // 32 lanes each start at a multiple of their width.
+  PredictArgs a = args;
+  for (int i = 1; i < a.n_win; ++i)
+    for (int j = i; j > 0 && a.windows[j] > a.windows[j - 1]; --j) {
+      const int t = a.windows[j];
+      a.windows[j] = a.windows[j - 1];
+      a.windows[j - 1] = t;
+    }
+  int sum = 0;
+  bool pow2 = true;
+  for (int i = 0; i < a.n_win; ++i) {
+    sum += a.windows[i];
+    pow2 = pow2 && a.windows[i] > 0 && (a.windows[i] & (a.windows[i] - 1)) == 0;
+  }
+  a.win_fast = (pow2 && sum <= 32) ? 1 : 0;
   return a.head_dim == 64 ? launch_d<64>(a, s) : launch_d<128>(a, s);
 }
 

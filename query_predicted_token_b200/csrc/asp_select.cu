@@ -5,7 +5,10 @@
 //
 // One 1024-thread CTA per row.  The row's 32-bit order keys live in shared
 // memory (up to 48K keys; longer rows are re-read from L2 in every sweep), so
-// no step needs another CTA.  Radix select from the most significant end with
+// no step needs another CTA.  When the first digit's histogram is given, the
+// threshold digit is found while the row's scores are still loading, and every
+// unit is classified and packed straight from registers: the row is read once
+// and no key array is built.  Radix select from the most significant end with
 // digits of 11, 11 and 10 bits: the first digit's histogram comes with the
 // scores (the key scan counts it with global atomics while it streams the
 // cache) or is built while the keys are loaded; later passes count only keys
@@ -29,6 +32,23 @@ constexpr int kSmemKeys = 48 * 1024;   // 192 KB of keys
 constexpr int kBins = kTopBins;        // widest digit: 11 bits
 constexpr int kBpt = kBins / kThreads;
 constexpr uint32_t kGtTag = 0x80000000u;
+
+// The float whose order key is k (see order_key), for a bin edge k: a NaN
+// pattern below the key of -inf gives -inf, one above the key of +inf gives NaN
+// (so that no score compares >= it).
+__device__ __forceinline__ float key_edge(uint32_t k) {
+  const uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+  if ((u & 0x7fffffffu) > 0x7f800000u) return (k & 0x80000000u) ? __uint_as_float(0x7fc00000u) : -INFINITY;
+  return __uint_as_float(u);
+}
+
+// A 16-byte load the compiler keeps in program order before later barriers, so
+// that every load of a thread is in flight before it waits at one.
+__device__ __forceinline__ float4 ld_issue(const float4* p) {
+  float4 v;
+  asm volatile("ld.global.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
+  return v;
+}
 
 // Exclusive scan of one int per thread over the CTA; also returns the total.
 __device__ __forceinline__ int cta_exclusive_scan(int x, int* wsum, int* total) {
@@ -66,7 +86,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   extern __shared__ __align__(16) uint32_t keys[];
   __shared__ int hist[2][kBins];
   __shared__ int wsum[kWarps];
-  __shared__ int wg[kWarps], we[kWarps], wn[kWarps];
+  __shared__ int wg[kWarps], we[kWarps];
   __shared__ int s_digit, s_above, s_bincnt, s_last_sel;
 
   int T = a.seq_lens ? a.seq_lens[b] : a.t_max;
@@ -108,8 +128,13 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
       if (lane == __ffs(peers) - 1) atomicAdd(&h[dig], __popc(peers));
     }
   };
-  if (cached && (a.row_stride & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0) {
-    const int n4 = (n + 3) >> 2;   // rows are 16-byte aligned: the last vector stays inside the row
+  // 16-byte rows: a row's last vector stays inside the row (row_stride is a multiple of 4)
+  const bool vec = (a.row_stride & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0;
+  // With the first histogram given, the threshold digit is found while the row's
+  // scores load, and the units are classified and packed straight from registers.
+  const bool fused = cached && !own_h0 && vec;
+  if (!fused && cached && vec) {
+    const int n4 = (n + 3) >> 2;
     constexpr int U = 4;           // vectors per thread in flight
     for (int base = 0; base < n4; base += U * kThreads) {
       float4 f[U];
@@ -129,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
         }
       }
     }
-  } else if (cached || own_h0) {
+  } else if (!fused && (cached || own_h0)) {
     for (int base = 0; base < n; base += kThreads) {
       const int i = base + tid;
       uint32_t key = 0u;
@@ -140,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
       if (own_h0) count_digit(h0, i < n, key >> kTopShift);
     }
   }
-  __syncthreads();
+  if (!fused) __syncthreads();
 
   // Finds the digit (of width nb) that holds the krem-th largest of the counted
   // keys, given this CTA's histogram h (or the row's global one).
@@ -182,16 +207,102 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     return done;
   };
 
-  // ---- first digit (11 bits)
-  bool done = find_digit(own_h0 ? h0 : a.hist0 + (size_t)row * kBins, 2048, kTopShift);
-  const uint32_t prefix0 = prefix, mask0 = mask;
-
-  // Warp w owns the contiguous units [w0, w1).
-  const int R = (((n + kWarps - 1) / kWarps) + 31) & ~31;
+  // Warp w owns the contiguous units [w0, w1) (in 128-unit chunks when fused).
+  const int R = fused ? ((((n + kWarps - 1) / kWarps) + 127) & ~127) : ((((n + kWarps - 1) / kWarps) + 31) & ~31);
   const int w0 = min(n, warp * R), w1 = min(n, w0 + R);
   const uint32_t lt_mask = (1u << lane) - 1u;
   int* h1 = hist[1];
   int n_packed = 0;
+  bool done;
+  uint32_t prefix0, mask0;
+  // Fused rows whose packed list fills at most half of the warp's range keep the
+  // candidates' keys at the range's end (entry k at w1 - 1 - k), so later passes
+  // need not re-read the scores.
+  bool kcache = false;
+  if (fused) {
+    // Lane l of a chunk holds units c0 + 4l .. c0 + 4l + 3 (one 16-byte load);
+    // four ballots give every surviving unit its packed position, in order.
+    constexpr int U = 8;   // chunks per warp in flight
+    const float4* s4 = reinterpret_cast<const float4*>(srow);
+    float4 f[U];
+    auto load_chunks = [&](int c0) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = c0 + u * 128 + 4 * lane;
+        f[u] = i < w1 ? ld_issue(s4 + (i >> 2)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    load_chunks(w0);
+    for (int i = tid; i < kBins; i += kThreads) h1[i] = 0;   // ordered by find_digit's barriers
+    done = find_digit(a.hist0 + (size_t)row * kBins, 2048, kTopShift);
+    prefix0 = prefix;
+    mask0 = mask;
+    // The bin's edges as floats: a unit survives (is above the bin or in it) iff
+    // score >= lo_f and is above it iff score >= hi_f.  An edge whose key is a NaN
+    // pattern lies beyond an infinity: below -inf every score passes, above +inf
+    // none does.  IEEE comparison already treats -0.0 as +0.0.
+    const uint32_t digit0 = prefix0 >> kTopShift;
+    const float lo_f = key_edge(prefix0);
+    const float hi_f = digit0 + 1u < (uint32_t)kBins ? key_edge((digit0 + 1u) << kTopShift) : __uint_as_float(0x7fc00000u);
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int c0 = w0; c0 < w1; c0 += U * 128) {
+      if (c0 != w0) load_chunks(c0);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = c0 + u * 128 + 4 * lane;
+        const float fv[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
+        bool sv[4], gt[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          sv[c] = i + c < w1 && fv[c] >= lo_f;
+          gt[c] = fv[c] >= hi_f;
+        }
+        // rank of unit (lane, c) among the chunk's survivors: all of the lower
+        // lanes' survivors, then this lane's earlier ones
+        uint32_t bs[4];
+        int before = 0, total = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          bs[c] = __ballot_sync(0xffffffffu, sv[c]);
+          before += __popc(bs[c] & lt);
+          total += __popc(bs[c]);
+        }
+        int pos = w0 + n_packed + before;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (sv[c]) keys[pos++] = (uint32_t)(i + c) | (gt[c] ? kGtTag : 0u);
+        n_packed += total;
+      }
+    }
+    __syncthreads();
+    kcache = 2 * n_packed <= w1 - w0;
+    if (!done) {   // the candidates' second digit, from the packed lists
+      constexpr int V = 4;   // entries per lane whose scores are in flight together
+      for (int k0 = 0; k0 < n_packed; k0 += 32 * V) {
+        uint32_t e[V];
+        float sc[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+          const int k = k0 + v * 32 + lane;
+          e[v] = k < n_packed ? keys[w0 + k] : kGtTag;
+          sc[v] = (e[v] & kGtTag) ? 0.f : srow[e[v]];
+        }
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+          const int k = k0 + v * 32 + lane;
+          const bool cand = !(e[v] & kGtTag);
+          const uint32_t key = order_key(sc[v]);
+          if (kcache && cand) keys[w1 - 1 - k] = key;
+          count_digit(h1, cand, (key >> 10) & 2047u);
+        }
+      }
+      __syncthreads();
+    }
+  } else {
+  // ---- first digit (11 bits)
+  done = find_digit(own_h0 ? h0 : a.hist0 + (size_t)row * kBins, 2048, kTopShift);
+  prefix0 = prefix;
+  mask0 = mask;
   if (cached) {
     // One sweep packs, in order and in place, every unit above the first-digit
     // threshold (tagged kGtTag) or inside its bin (a candidate), and counts the
@@ -222,10 +333,13 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     }
     __syncthreads();
   }
+  }
   // In the packed lists the tag bit marks units above the first-digit threshold;
-  // candidates' keys are re-read from the scores (they are few).
-  auto packed_key = [&](uint32_t e) -> uint32_t {
-    return (e & kGtTag) ? 0xffffffffu : order_key(srow[e & ~kGtTag]);
+  // candidates' keys come from the cache or are re-read from the scores (they
+  // are few).
+  auto packed_key = [&](uint32_t e, int k) -> uint32_t {
+    if (e & kGtTag) return 0xffffffffu;
+    return kcache ? keys[w1 - 1 - k] : order_key(srow[e]);
   };
 
   // ---- second (11 bits) and third (10 bits) digits
@@ -239,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
         for (int k0 = 0; k0 < n_packed; k0 += 32) {
           const int k = k0 + lane;
           const uint32_t e = k < n_packed ? keys[w0 + k] : kGtTag;
-          const uint32_t key = (e & kGtTag) ? 0u : packed_key(e);
+          const uint32_t key = (e & kGtTag) ? 0u : packed_key(e, k);
           count_digit(h2, !(e & kGtTag) && (key & mask) == prefix, key & 1023u);
         }
       } else {
@@ -261,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     if (!valid) return;
     if (cached) {
       if (e & kGtTag) { gt = true; return; }
-      const uint32_t mk = (mask == mask0) ? prefix0 : (packed_key(e) & mask);   // first digit alone: whole bin
+      const uint32_t mk = (mask == mask0) ? prefix0 : (packed_key(e, i - w0) & mask);   // first digit alone: whole bin
       gt = mk > prefix;
       eq = mk == prefix;
     } else {
