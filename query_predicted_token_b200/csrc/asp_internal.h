@@ -103,7 +103,7 @@ struct SelectArgs {
   int32_t* idx;
   int32_t* count;
   const int32_t* hist0;      // optional first-pass histogram [n_rows, 2048] (expand == 1 only)
-  int key_cap;               // set by launch_select: keys kept in shared memory per row (0 = none)
+  int key_cap;               // set by launch_select: shared-memory slots per row (keys, or packed lists)
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
 bool select_supported(int t_max, int expand);

@@ -8,7 +8,8 @@
 // no step needs another CTA.  When the first digit's histogram is given, the
 // threshold digit is found while the row's scores are still loading, and every
 // unit is classified and packed straight from registers: the row is read once
-// and no key array is built.  Radix select from the most significant end with
+// and no key array is built, so rows longer than the shared memory take this
+// path too (unless the survivors of the first digit overflow their slots).  Radix select from the most significant end with
 // digits of 11, 11 and 10 bits: the first digit's histogram comes with the
 // scores (the key scan counts it with global atomics while it streams the
 // cache) or is built while the keys are loaded; later passes count only keys
@@ -87,7 +88,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   __shared__ int hist[2][kBins];
   __shared__ int wsum[kWarps];
   __shared__ int wg[kWarps], we[kWarps];
-  __shared__ int s_digit, s_above, s_bincnt, s_last_sel;
+  __shared__ int s_digit, s_above, s_bincnt, s_last_sel, s_overflow;
 
   int T = a.seq_lens ? a.seq_lens[b] : a.t_max;
   T = T < 0 ? 0 : (T > a.t_max ? a.t_max : T);
@@ -110,9 +111,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     return;
   }
 
-  const bool cached = n <= a.key_cap;   // keys in shared memory, else re-read from L2
+  const bool cached = n <= a.key_cap;   // the whole row fits the shared-memory slots
   const float* srow = a.scores + (size_t)row * a.row_stride;
-  auto key_at = [&](int i) -> uint32_t { return cached ? keys[i] : order_key(srow[i]); };
 
   // ---- load the keys (cached rows) and, without a given first histogram, count the top digit
   const bool own_h0 = a.hist0 == nullptr;
@@ -132,7 +132,9 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   const bool vec = (a.row_stride & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0;
   // With the first histogram given, the threshold digit is found while the row's
   // scores load, and the units are classified and packed straight from registers.
-  const bool fused = cached && !own_h0 && vec;
+  const bool fused = !own_h0 && vec && a.key_cap >= kWarps * 4;
+  const bool keys_in_smem = cached && !fused;   // the key array is built (else keys are re-read from L2)
+  auto key_at = [&](int i) -> uint32_t { return keys_in_smem ? keys[i] : order_key(srow[i]); };
   if (!fused && cached && vec) {
     const int n4 = (n + 3) >> 2;
     constexpr int U = 4;           // vectors per thread in flight
@@ -211,13 +213,20 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   const int R = fused ? ((((n + kWarps - 1) / kWarps) + 127) & ~127) : ((((n + kWarps - 1) / kWarps) + 31) & ~31);
   const int w0 = min(n, warp * R), w1 = min(n, w0 + R);
   const uint32_t lt_mask = (1u << lane) - 1u;
+  // Warp w's packed list lives in the slots [pb, pe): its own range when the row
+  // fits, else an equal share of the slots (a longer list overflows it, and the
+  // row falls back to re-reading its scores in every pass).
+  const int share = (a.key_cap / kWarps) & ~3;
+  const int pb = (fused && !cached) ? warp * share : w0;
+  const int pe = (fused && !cached) ? pb + share : w1;
   int* h1 = hist[1];
   int n_packed = 0;
   bool done;
+  bool packed = cached;   // the packed lists hold every surviving unit
   uint32_t prefix0, mask0;
-  // Fused rows whose packed list fills at most half of the warp's range keep the
-  // candidates' keys at the range's end (entry k at w1 - 1 - k), so later passes
-  // need not re-read the scores.
+  // Packed lists that fill at most half of their slots keep the candidates' keys
+  // at the slots' end (entry k at pe - 1 - k), so later passes need not re-read
+  // the scores.
   bool kcache = false;
   if (fused) {
     // Lane l of a chunk holds units c0 + 4l .. c0 + 4l + 3 (one 16-byte load);
@@ -234,6 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     };
     load_chunks(w0);
     for (int i = tid; i < kBins; i += kThreads) h1[i] = 0;   // ordered by find_digit's barriers
+    if (tid == 0) s_overflow = 0;
     done = find_digit(a.hist0 + (size_t)row * kBins, 2048, kTopShift);
     prefix0 = prefix;
     mask0 = mask;
@@ -267,16 +277,21 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
           before += __popc(bs[c] & lt);
           total += __popc(bs[c]);
         }
-        int pos = w0 + n_packed + before;
+        if (n_packed + total <= pe - pb) {
+          int pos = pb + n_packed + before;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (sv[c]) keys[pos++] = (uint32_t)(i + c) | (gt[c] ? kGtTag : 0u);
+          for (int c = 0; c < 4; ++c)
+            if (sv[c]) keys[pos++] = (uint32_t)(i + c) | (gt[c] ? kGtTag : 0u);
+        } else if (lane == 0) {
+          s_overflow = 1;
+        }
         n_packed += total;
       }
     }
     __syncthreads();
-    kcache = 2 * n_packed <= w1 - w0;
-    if (!done) {   // the candidates' second digit, from the packed lists
+    packed = s_overflow == 0;
+    kcache = packed && 2 * n_packed <= pe - pb;
+    if (!done && packed) {   // the candidates' second digit, from the packed lists
       constexpr int V = 4;   // entries per lane whose scores are in flight together
       for (int k0 = 0; k0 < n_packed; k0 += 32 * V) {
         uint32_t e[V];
@@ -284,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
 #pragma unroll
         for (int v = 0; v < V; ++v) {
           const int k = k0 + v * 32 + lane;
-          e[v] = k < n_packed ? keys[w0 + k] : kGtTag;
+          e[v] = k < n_packed ? keys[pb + k] : kGtTag;
           sc[v] = (e[v] & kGtTag) ? 0.f : srow[e[v]];
         }
 #pragma unroll
@@ -292,9 +307,17 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
           const int k = k0 + v * 32 + lane;
           const bool cand = !(e[v] & kGtTag);
           const uint32_t key = order_key(sc[v]);
-          if (kcache && cand) keys[w1 - 1 - k] = key;
+          if (kcache && cand) keys[pe - 1 - k] = key;
           count_digit(h1, cand, (key >> 10) & 2047u);
         }
+      }
+      __syncthreads();
+    }
+    if (!done && !packed) {   // overflow: count the candidates from the scores
+      for (int base = 0; base < n; base += kThreads) {
+        const int i = base + tid;
+        const uint32_t key = i < n ? order_key(srow[i]) : 0u;
+        count_digit(h1, i < n && (key & mask0) == prefix0, (key >> 10) & 2047u);
       }
       __syncthreads();
     }
@@ -339,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   // are few).
   auto packed_key = [&](uint32_t e, int k) -> uint32_t {
     if (e & kGtTag) return 0xffffffffu;
-    return kcache ? keys[w1 - 1 - k] : order_key(srow[e]);
+    return kcache ? keys[pe - 1 - k] : order_key(srow[e]);
   };
 
   // ---- second (11 bits) and third (10 bits) digits
@@ -349,10 +372,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
       int* h2 = hist[0];
       for (int i = tid; i < 1024; i += kThreads) h2[i] = 0;
       __syncthreads();
-      if (cached) {
+      if (packed) {
         for (int k0 = 0; k0 < n_packed; k0 += 32) {
           const int k = k0 + lane;
-          const uint32_t e = k < n_packed ? keys[w0 + k] : kGtTag;
+          const uint32_t e = k < n_packed ? keys[pb + k] : kGtTag;
           const uint32_t key = (e & kGtTag) ? 0u : packed_key(e, k);
           count_digit(h2, !(e & kGtTag) && (key & mask) == prefix, key & 1023u);
         }
@@ -373,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   auto classify = [&](int i, uint32_t e, bool valid, bool& gt, bool& eq) {
     gt = eq = false;
     if (!valid) return;
-    if (cached) {
+    if (packed) {
       if (e & kGtTag) { gt = true; return; }
       const uint32_t mk = (mask == mask0) ? prefix0 : (packed_key(e, i - w0) & mask);   // first digit alone: whole bin
       gt = mk > prefix;
@@ -384,12 +407,12 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
       eq = mk == prefix;
     }
   };
-  const int span = cached ? n_packed : (w1 - w0);
+  const int span = packed ? n_packed : (w1 - w0);
   int c_gt = 0, c_eq = 0;
   for (int k0 = 0; k0 < span; k0 += 32) {
     const int k = k0 + lane;
     const bool valid = k < span;
-    const uint32_t e = (cached && valid) ? keys[w0 + k] : 0u;
+    const uint32_t e = (packed && valid) ? keys[pb + k] : 0u;
     bool gt, eq;
     classify(w0 + k, e, valid, gt, eq);
     c_gt += __popc(__ballot_sync(0xffffffffu, gt));
@@ -421,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   for (int k0 = 0; k0 < span; k0 += 32) {
     const int k = k0 + lane;
     const bool valid = k < span;
-    const uint32_t e = (cached && valid) ? keys[w0 + k] : 0u;
+    const uint32_t e = (packed && valid) ? keys[pb + k] : 0u;
     bool gt, eq;
     classify(w0 + k, e, valid, gt, eq);
     const uint32_t bg = __ballot_sync(0xffffffffu, gt);
@@ -429,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     const int Gj = run_gt + __popc(bg & lt_mask);
     const int Ej = run_eq + __popc(be & lt_mask);
     if (gt || (eq && Ej < krem)) {
-      const int u = cached ? (int)(e & ~kGtTag) : w0 + k;
+      const int u = packed ? (int)(e & ~kGtTag) : w0 + k;
       write_unit(u, Gj + min(Ej, krem));
       if (u == n - 1) s_last_sel = 1;
     }
@@ -447,7 +470,8 @@ bool select_supported(int t_max, int expand) { return t_max >= 1 && expand >= 1;
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   const int len_max = (a.t_max + a.expand - 1) / a.expand;
   SelectArgs args = a;
-  args.key_cap = len_max <= kSmemKeys ? ((len_max + 3) & ~3) : 0;   // same rule for every row
+  // shared-memory slots for keys or packed lists; the same for every row
+  args.key_cap = len_max <= kSmemKeys ? ((len_max + 3) & ~3) : kSmemKeys;
   const size_t smem = (size_t)(args.key_cap > 0 ? args.key_cap : 4) * 4;
   if (prepare_kernel((const void*)select_kernel, smem, kThreads) < 1) return cudaErrorInvalidConfiguration;
   return launch_pdl(select_kernel, dim3(args.n_rows), dim3(kThreads), smem, s, args);

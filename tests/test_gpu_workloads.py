@@ -165,3 +165,54 @@ def test_quest_page_scan_8b_32k():
         assert_valid_topk(ps[2, h].cpu().numpy(), npm, wl.C // P, pages, pages.size, "pages")
         ref_o, _ = oracle.attend_set(qg, keys[2][h], vals[2][h], sel)
         assert_out_close(out[2, h * G:(h + 1) * G], ref_o, torch.bfloat16, "quest attention")
+
+
+def _decode_once(k, v, lens, Hq, C, W=8, windows=(4, 8), seed=5):
+    """One decode step over a given cache; returns (scores, idx, count) of the new selection."""
+    B, Hkv, T, d = k.shape
+    g = torch.Generator().manual_seed(seed)
+    kv = asp.KV(k, v, lens.to(DEV), t_max=T)
+    qhist = torch.randn(B, Hq, W + 1, d, generator=g).to(DEV)
+    q_t = torch.randn(B, Hq, d, generator=g).to(k.dtype).to(DEV)
+    idx0, cnt0 = synth.random_selection(B, Hkv, C, lens.tolist(), seed=seed)
+    st = asp.DecodeState(kv, Hq, asp.PredCfg(W, windows, 1e-2), C, qhist.contiguous())
+    st.set_selection(idx0.to(DEV), cnt0.to(DEV))
+    out = torch.empty(B, Hq, d, dtype=k.dtype, device=DEV)
+    st.step(q_t, out)
+    assert asp.wait_selection(st.ev_sel_done, 60_000_000) == 0
+    torch.cuda.synchronize()
+    assert asp.device_status() == 0
+    idx1, cnt1 = (t.cpu().numpy() for t in st.selection)
+    return st.scores.cpu().numpy(), idx1, cnt1
+
+
+def test_decode_selection_of_tied_scores_keeps_the_first_tokens():
+    """Zero keys make every score equal: each row keeps its first C tokens.  The rows
+    span every path of the selection: shorter than C, fitting its shared memory, and
+    longer than that (where the packed lists of all-tied rows overflow)."""
+    B, Hkv, G, d, T, C = 4, 2, 2, 128, 65536, 2048
+    lens = torch.tensor([1000, 30000, 50000, 65536], dtype=torch.int32)
+    k = torch.zeros(B, Hkv, T, d, dtype=torch.bfloat16, device=DEV)
+    v = torch.zeros(B, Hkv, T, d, dtype=torch.bfloat16, device=DEV)
+    scores, idx, cnt = _decode_once(k, v, lens, Hkv * G, C)
+    for b in range(B):
+        n = min(C, int(lens[b]))
+        for h in range(Hkv):
+            assert np.all(scores[b, h, :lens[b]] == 0.0)
+            assert int(cnt[b, h]) == n
+            assert idx[b, h, :n].tolist() == list(range(n)), f"b{b}h{h}"
+            assert np.all(idx[b, h, n:] == -1)
+
+
+def test_decode_selection_when_most_tokens_survive_the_first_digit():
+    """C close to T_b on rows longer than the selection's shared memory: the survivors
+    of the first digit overflow the packed lists and the row is re-read from L2."""
+    B, Hkv, G, d, T, C = 2, 2, 2, 128, 60000, 50000
+    lens = torch.tensor([60000, 52000], dtype=torch.int32)
+    g = torch.Generator().manual_seed(7)
+    k = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).to(DEV)
+    v = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).to(DEV)
+    scores, idx, cnt = _decode_once(k, v, lens, Hkv * G, C)
+    for b in range(B):
+        for h in range(Hkv):
+            assert_valid_topk(scores[b, h], int(lens[b]), C, idx[b, h], int(cnt[b, h]), f"b{b}h{h}")
