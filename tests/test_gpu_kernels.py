@@ -86,6 +86,61 @@ def test_score_keys(dtype, d, G, page_size):
             assert np.isnan(got[b, h, Tb:]).all()      # entries past T_b are not written
 
 
+_MANY_SHORT = [int(x) for x in np.random.default_rng(3).integers(1, 41, 200)]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("lens", [[1000, 530, 17], _MANY_SHORT], ids=["three", "many_short"])
+def test_score_keys_whole_pages(d, G, lens):
+    """8 KV heads in 16-token pages: one tile per page of every head.  200 short
+    sequences make every CTA switch sequences within a few tiles."""
+    B, Hkv = len(lens), 8
+    T = max(lens)
+    kvd, kv = make_cache(B, Hkv, d, T, torch.bfloat16, lens, 16, seed=G + d)
+    qpred = torch.randn(B, Hkv * G, d, generator=_gen(6)).to(DEV)
+    scores = torch.full((B, Hkv, T), float("nan"), device=DEV)
+    asp.score_keys(qpred, kv, scores)
+    torch.cuda.synchronize()
+    keys, _ = host_sequences(kvd)
+    ref = oracle.score_keys(np64(qpred), [keys[b] for b in range(B)], T)
+    got = scores.cpu().numpy()
+    for b in range(B):
+        for h in range(Hkv):
+            Tb = lens[b]
+            assert_scores_close(got[b, h, :Tb], ref[b, h, :Tb], np64(qpred[b, h * G:(h + 1) * G]), keys[b][h],
+                                what=f"b{b} h{h}")
+            assert np.isnan(got[b, h, Tb:]).all()
+
+
+def test_decode_step_on_whole_pages_selects_the_top_scores():
+    """The decode step on a paged cache of 8 KV heads (GQA group 8, d = 64): the
+    selection, made from the histogram the page scan counts, is the top C of the
+    step's own scores, and the scores match the oracle."""
+    lens = [3000, 5000, 700, 4100]
+    B, Hkv, G, d, C, W = len(lens), 8, 8, 64, 256, 8
+    kvd, kv = make_cache(B, Hkv, d, max(lens), torch.bfloat16, lens, 16, seed=12)
+    g = _gen(13)
+    qhist = torch.randn(B, Hkv * G, W + 1, d, generator=g).to(DEV).contiguous()
+    q_t = torch.randn(B, Hkv * G, d, generator=g).to(torch.bfloat16).to(DEV)
+    idx0, cnt0 = random_selection(B, Hkv, C, lens, seed=14)
+    st = asp.DecodeState(kv, Hkv * G, asp.PredCfg(W, (4, 8), 1e-2), C, qhist)
+    st.set_selection(idx0.to(DEV), cnt0.to(DEV))
+    out = torch.empty(B, Hkv * G, d, dtype=torch.bfloat16, device=DEV)
+    st.step(q_t, out)
+    assert asp.wait_selection(st.ev_sel_done, 60_000_000) == 0
+    torch.cuda.synchronize()
+    scores = st.scores.cpu().numpy()
+    idx1, cnt1 = (t.cpu().numpy() for t in st.selection)
+    keys, _ = host_sequences(kvd)
+    pred = st.qpred.cpu().double().numpy()
+    for b in range(B):
+        for h in range(Hkv):
+            assert_valid_topk(scores[b, h], lens[b], C, idx1[b, h], int(cnt1[b, h]), f"b{b}h{h}")
+            ref = oracle.score_row(pred[b, h * G:(h + 1) * G], keys[b][h])
+            assert_scores_close(scores[b, h, :lens[b]], ref, pred[b, h * G:(h + 1) * G], keys[b][h], f"b{b}h{h}")
+
+
 def test_score_empty_sequence_writes_nothing():
     kvd, kv = make_cache(2, 2, 128, 64, torch.bfloat16, [0, 40])
     qpred = torch.randn(2, 8, 128, generator=_gen(1)).to(DEV)

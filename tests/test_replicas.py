@@ -57,12 +57,16 @@ def _rank_main(rank: int, world: int, port: int, q) -> None:
 
 
 def _rank_dies(rank: int, world: int, port: int, q) -> None:
-    """Rank 1 raises after joining; rank 0 then enters a collective."""
+    """Rank 1 exits abruptly after joining (no teardown, so its sockets close at
+    once); rank 0 then enters a collective."""
     _rank_env(rank, world, port)
     g = ReplicaGroup("gloo", "cpu", timeout_s=5)
+    g.barrier()   # both ranks fully connected before one of them leaves
     if rank == 1:
         q.put((rank, "raised", None))
-        raise SystemExit(3)
+        q.close()
+        q.join_thread()   # the message is out before the process ends
+        os._exit(3)
     try:
         g.slowest(1.0)
         q.put((rank, "no error", None))
