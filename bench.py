@@ -41,6 +41,7 @@ def parse():
     ap.add_argument("--workload", default="qwen3_8b_shaped_32k")
     ap.add_argument("--impl", default="asp", choices=["asp", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-compare", action="store_true", help="skip the page-level and full-attention timings")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
 
@@ -58,6 +59,31 @@ def step_bytes(wl, lens):
     attend = sel_units * d * e * 2 + B * Hq * d * (e + e + 4) + B * Hkv * C * 4
     return dict(predict=predict, score=score, select=select, attend=attend,
                 total=predict + score + select + attend)
+
+
+QUEST_PAGE = 16
+
+
+def quest_step_bytes(wl, lens):
+    """Algorithmic HBM bytes of one step of the page-level comparison path: the
+    per-page key bounds (min and max rows), the page scores written and read back,
+    the chosen pages' indices, and the attention over the chosen tokens."""
+    e = 2 if wl.kv_dtype == "bf16" else 4
+    B, Hq, Hkv, d, C = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.C
+    pages = sum(math.ceil(int(t) / QUEST_PAGE) for t in lens) * Hkv
+    cp = math.ceil(C / QUEST_PAGE) * QUEST_PAGE
+    scan = pages * 2 * d * e + pages * 4 + B * Hq * d * e
+    select = pages * 4 + B * Hkv * cp * 4
+    sel_units = sum(min(cp, int(t)) for t in lens) * Hkv
+    attend = sel_units * d * e * 2 + B * Hq * d * (e + e) + B * Hkv * cp * 4
+    return dict(scan=scan, select=select, attend=attend, total=scan + select + attend)
+
+
+def dense_bytes(wl, lens):
+    """Full attention over every cached token: every K and V row once."""
+    e = 2 if wl.kv_dtype == "bf16" else 4
+    tok = sum(int(t) for t in lens)
+    return tok * wl.n_kv_heads * wl.head_dim * e * 2 + wl.batch * wl.n_q_heads * wl.head_dim * (e + e)
 
 
 def read_peaks():
@@ -238,6 +264,60 @@ def run_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- comparison paths
+def comparison_paths(wl, kvd, kv, q_dev, stream, flush, steps):
+    """Times, on the same cache and query, the page-level comparison path (page
+    bound scan and page choice with the current query, then attention over the
+    chosen pages' tokens) and full attention over every cached token.  The page
+    bounds are built once beforehand (a serving system keeps them up to date as
+    tokens arrive).  Returns a dict for the JSON line."""
+    import torch
+    import query_predicted_token_b200 as asp
+    B, Hq, Hkv, d, C = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.C
+    dev = kvd["k"].device
+    lens = kvd["seq_lens"].cpu().tolist()
+    npm = math.ceil(wl.t_max / QUEST_PAGE)
+    cp = math.ceil(C / QUEST_PAGE) * QUEST_PAGE
+    meta = torch.empty(B, Hkv, npm, 2, d, dtype=wl.torch_dtype(), device=dev)
+    ps = torch.empty(B, Hkv, npm, device=dev)
+    qidx = torch.empty(B, Hkv, cp, dtype=torch.int32, device=dev)
+    qcnt = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
+    out = torch.empty(B, Hq, d, dtype=wl.torch_dtype(), device=dev)
+    ws_q = torch.empty(max(16, asp.attend_workspace_bytes(B, Hq, Hkv, d, cp)), dtype=torch.uint8, device=dev)
+    zero = torch.zeros(B, dtype=torch.int32, device=dev)
+    ws_d = torch.empty(max(16, asp.attend_workspace_bytes(B, Hq, Hkv, d, 0, wl.t_max)), dtype=torch.uint8,
+                       device=dev)
+    with torch.cuda.stream(stream):
+        asp.quest_build_meta(kv, QUEST_PAGE, meta, stream=stream)
+
+    def quest_step():
+        asp.quest_select(q_dev, kv, meta, QUEST_PAGE, C, ps, qidx, qcnt, stream=stream)
+        asp.sparse_attend(q_dev, kv, qidx, qcnt, cp, out, workspace=ws_q, stream=stream)
+
+    def dense_step():
+        asp.sparse_attend(q_dev, kv, None, None, 0, out, None, zero, wl.t_max, ws_d, stream=stream)
+
+    res = {}
+    for name, fn, nbytes in (("page_level", quest_step, quest_step_bytes(wl, lens)["total"]),
+                             ("full_attention", dense_step, dense_bytes(wl, lens))):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        with torch.cuda.stream(stream):
+            for k in range(-3, steps):
+                flush.zero_()
+                if k >= 0:
+                    ev[k][0].record(stream)
+                fn()
+                if k >= 0:
+                    ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+        res[name] = {"step_us": round(ms * 1e3, 2), "gbs": round(nbytes / (ms / 1e3) / 1e9, 1), "bytes": nbytes}
+    res["note"] = ("same cache, query and L2 flush; page_level: page bounds scanned with the current query, "
+                   f"{cp // QUEST_PAGE} pages of {QUEST_PAGE} kept, attention over their tokens; "
+                   "full_attention: every cached token")
+    return res
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def main():
     args = parse()
@@ -328,6 +408,8 @@ def main():
         one_step(k, e2e=True)
     torch.cuda.synchronize()
     e2e_ms = [a.elapsed_time(b) for a, b in ev]
+    # the pages' two baselines on the same cache and query: page-level selection, full attention
+    compare = None if args.no_compare else comparison_paths(wl, kvd, kv, q_t, s_main, flush, args.steps)
 
     t_rank, t_e2e = group.slowest(sum(step_ms) / 1e3, sum(e2e_ms) / 1e3)
     (total_bytes,) = group.total(acct["total"] * args.steps)   # ragged batches differ per rank
@@ -368,6 +450,7 @@ def main():
                     "d2h_bytes_per_step": out.numel() * out.element_size()},
             "gpu_launches": args.steps * (4 + (1 if splits else 0)),
             "cpu_baseline": cpu,
+            "comparison": compare,
         }
         print(json.dumps(line), flush=True)
     group.close()

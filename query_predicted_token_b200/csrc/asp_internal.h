@@ -83,6 +83,9 @@ cudaError_t launch_score(const float* qpred, int n_q_heads, const KvView& kv, fl
 
 // Tensor-core key scan (bf16 keys, head_dim 64/128, contiguous or 16-token pages,
 // G in {1,2,4,8}, 16-byte aligned qpred); launch_score uses it when supported.
+bool quest_tc_supported(const KvView& kv, int n_q_heads, const void* q);
+cudaError_t launch_quest_score_tc(const void* q, int q_f32, int n_q_heads, const KvView& kv, const void* meta,
+                                  int quest_page, float* page_scores, cudaStream_t s);
 bool score_tc_supported(const KvView& kv, int n_q_heads, const float* qpred);
 cudaError_t launch_score_tc(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s,
                             int32_t* hist);

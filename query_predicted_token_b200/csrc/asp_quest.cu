@@ -212,6 +212,8 @@ cudaError_t launch_quest_meta(const KvView& kv, int quest_page, void* meta, cuda
 
 cudaError_t launch_quest_score(const void* q, int q_f32, int n_q_heads, const KvView& kv, const void* meta,
                                int quest_page, float* page_scores, cudaStream_t s) {
+  if (quest_tc_supported(kv, n_q_heads, q))   // bf16 bounds: on the tensor cores
+    return launch_quest_score_tc(q, q_f32, n_q_heads, kv, meta, quest_page, page_scores, s);
   const int G = n_q_heads / kv.n_kv;
   if (kv.kv_f32) {
     return kv.head_dim == 64 ? score_g<float, 64>(G, q, q_f32, n_q_heads, kv, meta, quest_page, page_scores, s)

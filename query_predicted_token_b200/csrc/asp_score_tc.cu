@@ -32,6 +32,8 @@ namespace {
 constexpr int kTileT = 128;    // tokens per tile = MMA M
 constexpr int kN = 16;         // MMA N: rows (hi, lo) of the group's queries, padded
 constexpr int kStages = 4;
+// stages of the token-tile ring: three 64 KB tiles for 256-channel rows
+__host__ __device__ constexpr int stages_for(int D) { return D >= 256 ? 3 : kStages; }
 constexpr int kThreadsTC = 192;
 constexpr uint32_t kTmemCols = 32;   // two 16-column fp32 accumulators
 // instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major, N, M
@@ -40,6 +42,12 @@ constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kN 
 
 struct TcParams {
   const float* qpred;
+  // page-bound mode: each "key" row is a page's [kmin, kmax] (2d channels) and
+  // each query row is [min(q, 0), max(q, 0)], so the dot product is the bound
+  const void* qraw;   // the current query (bf16 or fp32) in page-bound mode, else null
+  int qraw_f32;
+  int len_div;        // units per length: 1 for tokens, the page size for page bounds
+  int len_cap;        // cap of seq_lens (tokens)
   int n_q_heads, G;   // G is also the kernel's template argument
   int batch, n_kv, t_max, page_size, max_pages, n_pages;
   const int32_t* page_table;
@@ -160,6 +168,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_co
   constexpr int STAGE = KBYTES + QBYTES;              // multiple of 1024
   constexpr int KSTEPS = D / 16;
   constexpr int QCH = HALVES * kN * 8 / 32;           // 16-byte Q chunks per producer lane
+  constexpr int kStages = stages_for(D);
   static_assert(STAGE % 1024 == 0, "stage alignment");
 
   extern __shared__ uint8_t smem_raw[];
@@ -198,8 +207,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_co
   pdl_wait();
   pdl_trigger();   // the selection may launch while the scan runs
   for (int b = threadIdx.x; b < p.batch; b += blockDim.x) {
-    int t = p.seq_lens ? p.seq_lens[b] : p.t_max;
-    lens[b] = t < 0 ? 0 : (t > p.t_max ? p.t_max : t);
+    int t = p.seq_lens ? p.seq_lens[b] : p.len_cap;
+    t = t < 0 ? 0 : (t > p.len_cap ? p.len_cap : t);
+    lens[b] = (t + p.len_div - 1) / p.len_div;   // rows of this sequence
   }
   __syncthreads();
   cta_prefix_sum(p.batch, pre, [&](int b) { return ((lens[b] + kTileT - 1) / kTileT) * p.n_kv; }, scratch);
@@ -269,10 +279,35 @@ __global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_co
           for (int e = 0; e < 8; ++e) x[e] = 0.f;
           const int g = r < G ? r : r - G;
           if (r < 2 * G) {
-            const float* src = p.qpred + ((size_t)(c.b * p.n_q_heads + c.h * G + g)) * D + half * 64 + col * 8;
-            const float4 a0 = *reinterpret_cast<const float4*>(src);
-            const float4 a1 = *reinterpret_cast<const float4*>(src + 4);
-            const float v[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            float v[8];
+            if (p.qraw) {   // page bounds: [min(q, 0), max(q, 0)] of the current query
+              constexpr int DQ = D / 2;
+              const int ch = half * 64 + col * 8;
+              const size_t off = (size_t)(c.b * p.n_q_heads + c.h * G + g) * DQ + (ch < DQ ? ch : ch - DQ);
+              if (p.qraw_f32) {
+                const float4 a0 = *reinterpret_cast<const float4*>(static_cast<const float*>(p.qraw) + off);
+                const float4 a1 = *reinterpret_cast<const float4*>(static_cast<const float*>(p.qraw) + off + 4);
+                v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w;
+                v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
+              } else {
+                const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.qraw) + off);
+                float2 f[4];
+                Elem<__nv_bfloat16>::unpack(u, f);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  v[2 * e] = f[e].x;
+                  v[2 * e + 1] = f[e].y;
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[e] = ch < DQ ? fminf(v[e], 0.f) : fmaxf(v[e], 0.f);
+            } else {
+              const float* src = p.qpred + ((size_t)(c.b * p.n_q_heads + c.h * G + g)) * D + half * 64 + col * 8;
+              const float4 a0 = *reinterpret_cast<const float4*>(src);
+              const float4 a1 = *reinterpret_cast<const float4*>(src + 4);
+              v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w;
+              v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
+            }
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const float q = v[e] * p.scale;
@@ -717,7 +752,8 @@ cudaError_t launch_tc_t(const KvView& kv, const TcParams& p, cudaStream_t s) {
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   constexpr int STAGE = kTileT * D * 2 + (D / 64) * kN * 128;
-  const size_t smem = 1024 + (size_t)kStages * STAGE + (2 * kStages + 4) * 8 + (2 * (size_t)p.batch + 1) * 4;
+  constexpr int S = stages_for(D);
+  const size_t smem = 1024 + (size_t)S * STAGE + (2 * S + 4) * 8 + (2 * (size_t)p.batch + 1) * 4;
   auto kern = score_tc_kernel<D, G>;
   if (prepare_kernel((const void*)kern, smem, kThreadsTC) < 1) return cudaErrorInvalidConfiguration;
   return launch_pdl(kern, dim3(sm_count()), dim3(kThreadsTC), smem, s, map, p);
@@ -758,6 +794,10 @@ cudaError_t launch_score_tc(const float* qpred, int n_q_heads, const KvView& kv,
                             int32_t* hist) {
   TcParams p;
   p.qpred = qpred;
+  p.qraw = nullptr;
+  p.qraw_f32 = 0;
+  p.len_div = 1;
+  p.len_cap = kv.t_max;
   p.n_q_heads = n_q_heads;
   p.G = n_q_heads / kv.n_kv;
   p.batch = kv.batch;
@@ -793,6 +833,53 @@ cudaError_t launch_score_tc(const float* qpred, int n_q_heads, const KvView& kv,
     case -2: return launch_tc_t<128, 2>(kv, p, s);
     case -4: return launch_tc_t<128, 4>(kv, p, s);
     case -8: return launch_tc_t<128, 8>(kv, p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Page bounds on the tensor cores: meta [batch, n_kv, npm, 2, d] read as a
+// contiguous cache of 2d-channel rows, one row per page.
+bool quest_tc_supported(const KvView& kv, int n_q_heads, const void* q) {
+  const int G = n_q_heads / kv.n_kv;
+  return !kv.kv_f32 && (kv.head_dim == 64 || kv.head_dim == 128) && (G == 1 || G == 2 || G == 4 || G == 8) &&
+         kv.batch <= 1024 && (reinterpret_cast<uintptr_t>(q) & 15) == 0;
+}
+
+cudaError_t launch_quest_score_tc(const void* q, int q_f32, int n_q_heads, const KvView& kv, const void* meta,
+                                  int quest_page, float* page_scores, cudaStream_t s) {
+  const int npm = (kv.t_max + quest_page - 1) / quest_page;
+  TcParams p;
+  p.qpred = nullptr;
+  p.qraw = q;
+  p.qraw_f32 = q_f32;
+  p.len_div = quest_page;
+  p.len_cap = kv.t_max;
+  p.n_q_heads = n_q_heads;
+  p.G = n_q_heads / kv.n_kv;
+  p.batch = kv.batch;
+  p.n_kv = kv.n_kv;
+  p.t_max = npm;   // rows per (sequence, head) in meta, and the page scores' row stride
+  p.page_size = 0;
+  p.max_pages = 0;
+  p.n_pages = 0;
+  p.page_table = nullptr;
+  p.seq_lens = kv.seq_lens;
+  p.scores = page_scores;
+  p.hist = nullptr;
+  p.scale = 1.0f / sqrtf((float)kv.head_dim);
+  KvView mv = kv;   // the tensor map's view: rows of meta
+  mv.k = meta;
+  mv.page_size = 0;
+  mv.t_max = npm;
+  switch (p.G * (kv.head_dim == 64 ? 1 : -1)) {
+    case 1: return launch_tc_t<128, 1>(mv, p, s);
+    case 2: return launch_tc_t<128, 2>(mv, p, s);
+    case 4: return launch_tc_t<128, 4>(mv, p, s);
+    case 8: return launch_tc_t<128, 8>(mv, p, s);
+    case -1: return launch_tc_t<256, 1>(mv, p, s);
+    case -2: return launch_tc_t<256, 2>(mv, p, s);
+    case -4: return launch_tc_t<256, 4>(mv, p, s);
+    case -8: return launch_tc_t<256, 8>(mv, p, s);
     default: return cudaErrorInvalidValue;
   }
 }
