@@ -122,8 +122,13 @@ asp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ASP_OK : ASP_E
 
 // asp_decode_step's workspace: the attention's split-K partials, then (256-byte
 // aligned) the key-score histogram [batch * n_kv, 2048] int32 of the selection.
+// The decode step's attention runs beside the selection chain: one CTA per SM
+// leaves room for the key scan's CTA on every SM.
+constexpr int kDecodeAttendCtasPerSm = 1;
+
 size_t decode_hist_offset(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail) {
-  const size_t att = asp::attend_plan(batch, n_q_heads, n_kv_heads, head_dim, C, max_tail).workspace_bytes;
+  const size_t att =
+      asp::attend_plan(batch, n_q_heads, n_kv_heads, head_dim, C, max_tail, kDecodeAttendCtasPerSm).workspace_bytes;
   return ((att + 255) / 256) * 256;
 }
 
@@ -154,7 +159,7 @@ asp::PredictArgs predict_args(float* qhist, int ring_start, const void* q_new, a
 
 asp_status check_attend(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv, const int32_t* idx,
                         const int32_t* count, int C, const int32_t* tail_begin, int max_tail, void* out,
-                        void* workspace, size_t workspace_bytes, asp::AttendPlan* plan) {
+                        void* workspace, size_t workspace_bytes, asp::AttendPlan* plan, int ctas_per_sm = 0) {
   asp_status st = check_kv(kv, true);
   if (st != ASP_OK) return st;
   if (!q || !out) return ASP_ERR_INVALID_ARG;
@@ -165,7 +170,7 @@ asp_status check_attend(const void* q, asp_dtype q_dtype, int n_q_heads, const a
   const int mt = tail_begin ? max_tail : 0;
   if (mt < 0 || (long)C + mt < 1) return ASP_ERR_INVALID_ARG;
   if ((long)C + mt > (1L << 30)) return ASP_ERR_UNSUPPORTED;
-  *plan = asp::attend_plan(kv->batch, n_q_heads, kv->n_kv_heads, kv->head_dim, C, mt);
+  *plan = asp::attend_plan(kv->batch, n_q_heads, kv->n_kv_heads, kv->head_dim, C, mt, ctas_per_sm);
   if (plan->workspace_bytes) {
     if (!workspace || workspace_bytes < plan->workspace_bytes) return ASP_ERR_WORKSPACE;
     if (!aligned16(workspace)) return ASP_ERR_WORKSPACE;
@@ -279,7 +284,7 @@ asp_status asp_decode_step(const asp_decode_args* a) {
   if (!a) return ASP_ERR_INVALID_ARG;
   asp::AttendPlan plan;
   asp_status st = check_attend(a->q_t, a->q_dtype, a->n_q_heads, a->kv, a->idx_cur, a->count_cur, a->C, a->tail_begin,
-                               a->max_tail, a->out, a->workspace, a->workspace_bytes, &plan);
+                               a->max_tail, a->out, a->workspace, a->workspace_bytes, &plan, kDecodeAttendCtasPerSm);
   if (st != ASP_OK) return st;
   if (a->C < 1 || !a->qhist || !a->qpred || !a->scores || !a->idx_next || !a->count_next) return ASP_ERR_INVALID_ARG;
   const int mt = a->tail_begin ? a->max_tail : 0;
@@ -318,7 +323,9 @@ asp_status asp_decode_step(const asp_decode_args* a) {
   }
   if (e == cudaSuccess) e = mark(1, ss);
   if (e == cudaSuccess) e = mark(2, ss);
-  if (e == cudaSuccess) e = asp::launch_score(a->qpred, a->n_q_heads, kv, a->scores, ss, hist);
+  // the predictor is the scan's only producer in this stream: the scan may start
+  // streaming keys while it runs
+  if (e == cudaSuccess) e = asp::launch_score(a->qpred, a->n_q_heads, kv, a->scores, ss, hist, true);
   if (e == cudaSuccess) e = mark(3, ss);
   if (e == cudaSuccess) e = mark(4, ss);
   if (e == cudaSuccess) {

@@ -780,16 +780,17 @@ cudaError_t dispatch_g(int G, const AttParams& p, cudaStream_t s) {
 }  // namespace
 
 // Split plan: as many splits per KV head as fit in one wave of resident CTAs on
-// a 148-SM B200 (3 CTAs per SM for G <= 4, 2 for G = 8, set by the registers),
-// each split a multiple of 64 rows (one 16-row tile per warp).  A pure function
-// of the sizes, so the workspace size is known without a device.
-AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail) {
+// a 148-SM B200 (by default 3 CTAs per SM for G <= 4, 2 for G = 8, set by the
+// registers), each split a multiple of 64 rows (one 16-row tile per warp).  A
+// pure function of the sizes, so the workspace size is known without a device.
+AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail,
+                       int ctas_per_sm) {
   AttendPlan pl{1, 64, 0};
   const long rows = (long)C + (max_tail > 0 ? max_tail : 0);
   const long units = (long)batch * n_kv_heads;
   if (rows <= 0 || units <= 0 || n_kv_heads <= 0) return pl;
   const int G = n_q_heads / n_kv_heads;
-  const long target = 148L * (G >= 8 ? 2 : 3);
+  const long target = 148L * (ctas_per_sm > 0 ? ctas_per_sm : (G >= 8 ? 2 : 3));
   const int quantum = kTile * kWarps;
   long splits = target / units;
   if (splits < 1) splits = 1;

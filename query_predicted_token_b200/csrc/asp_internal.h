@@ -78,8 +78,11 @@ struct KvView {
 };
 // hist: optional [batch * n_kv, 2048] int32 counts of the scores' top 11 key bits
 // (must be zero on entry); the selection then skips its own first pass.
+// early: the previous kernel of the stream writes only qpred (and clears hist), and
+// every other input was written before it started; the tensor-core scan then
+// starts streaming keys before that kernel has finished.
 cudaError_t launch_score(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s,
-                         int32_t* hist = nullptr);
+                         int32_t* hist = nullptr, bool early = false);
 
 // Tensor-core key scan (bf16 keys, head_dim 64/128, contiguous or 16-token pages,
 // G in {1,2,4,8}, 16-byte aligned qpred); launch_score uses it when supported.
@@ -88,7 +91,7 @@ cudaError_t launch_quest_score_tc(const void* q, int q_f32, int n_q_heads, const
                                   int quest_page, float* page_scores, cudaStream_t s);
 bool score_tc_supported(const KvView& kv, int n_q_heads, const float* qpred);
 cudaError_t launch_score_tc(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s,
-                            int32_t* hist);
+                            int32_t* hist, bool early = false);
 
 // ---- step 3 -----------------------------------------------------------------
 // Selects `c_units` units per row out of ceil(T_b / expand) scores (row stride
@@ -117,7 +120,9 @@ struct AttendPlan {
   int rows_per_split;
   size_t workspace_bytes;
 };
-AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail);
+// ctas_per_sm: resident CTAs per SM the grid is sized for (0: as many as fit).
+AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail,
+                       int ctas_per_sm = 0);
 cudaError_t launch_attend(const void* q, int q_f32, int n_q_heads, const KvView& kv, const int32_t* idx,
                           const int32_t* count, int C, const int32_t* tail_begin, int max_tail, void* out,
                           float* lse, void* workspace, const AttendPlan& plan, cudaStream_t s);

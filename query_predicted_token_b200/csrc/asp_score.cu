@@ -277,8 +277,8 @@ cudaError_t dispatch_g(int G, const ScoreParams& p, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_score(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s,
-                         int32_t* hist) {
-  if (score_tc_supported(kv, n_q_heads, qpred)) return launch_score_tc(qpred, n_q_heads, kv, scores, s, hist);
+                         int32_t* hist, bool early) {
+  if (score_tc_supported(kv, n_q_heads, qpred)) return launch_score_tc(qpred, n_q_heads, kv, scores, s, hist, early);
   ScoreParams p;
   p.qpred = qpred;
   p.n_q_heads = n_q_heads;

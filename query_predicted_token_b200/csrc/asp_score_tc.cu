@@ -48,6 +48,7 @@ struct TcParams {
   int qraw_f32;
   int len_div;        // units per length: 1 for tokens, the page size for page bounds
   int len_cap;        // cap of seq_lens (tokens)
+  int early;          // stream the first tiles' keys before the previous kernel ends
   int n_q_heads, G;   // G is also the kernel's template argument
   int batch, n_kv, t_max, page_size, max_pages, n_pages;
   const int32_t* page_table;
@@ -203,9 +204,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_co
   }
   // Everything above touches no global memory, so it overlaps the previous
   // kernel; the predicted queries, the cleared histogram and the cache
-  // description are read only after it has finished.
-  pdl_wait();
-  pdl_trigger();   // the selection may launch while the scan runs
+  // description are read only after it has finished.  In early mode that kernel
+  // writes nothing else, so the cache description is read at once and the
+  // producer streams its first tiles' keys before it waits.
+  const bool early = p.early && p.page_size == 0;
+  if (!early) pdl_wait();
   for (int b = threadIdx.x; b < p.batch; b += blockDim.x) {
     int t = p.seq_lens ? p.seq_lens[b] : p.len_cap;
     t = t < 0 ? 0 : (t > p.len_cap ? p.len_cap : t);
@@ -217,6 +220,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
+  if (early && warp != 0) pdl_wait();
+  pdl_trigger();   // the selection may launch while the scan runs
 
   const int total = pre[p.batch];
   const int chunk = (total + gridDim.x - 1) / gridDim.x;
@@ -260,6 +265,22 @@ __global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_co
     uint4 qreg[QCH];
     int pt_b = -1, pt_base = 0, pt_val = -1, pt_next = -1;
     int issued = 0, done_ok = 1;
+    int pre_k = 0;   // tiles whose keys were requested before the wait
+    if (early) {
+      TileCursor pc;
+      locate(t0, pc);
+      pre_k = min(kStages, n_my);
+      for (int k = 0; k < pre_k; ++k) {
+        if (lane == 0) mbar_expect_tx(&full[k], KBYTES);
+        __syncwarp();
+        if (lane < HALVES) {
+          const int y = (pc.b * p.n_kv + pc.h) * p.t_max + pc.tile * kTileT;
+          tma_load_2d(sbase + k * STAGE + lane * (kTileT * 128), &kmap, lane * 64, y, &full[k], policy);
+        }
+        advance(pc);
+      }
+      pdl_wait();
+    }
     for (int k = 0; k < n_my; ++k) {
       const int s = k % kStages;
       const uint32_t ph = (uint32_t)(k / kStages) & 1u;
@@ -328,6 +349,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_co
       }
       fence_proxy_async_smem();
       __syncwarp();
+      if (k < pre_k) {   // the keys are on their way: only the queries were missing
+        if (lane == 0) mbar_arrive(&full[s]);
+        ++issued;
+        advance(c);
+        continue;
+      }
       if (lane == 0) mbar_arrive_expect_tx(&full[s], KBYTES);
       __syncwarp();
       const uint32_t sdst = sbase + s * STAGE;
@@ -370,7 +397,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_co
       advance(c);
     }
     if (!done_ok) {   // a wait ran out: give the copies in flight a bounded chance to land
-      for (int k = max(0, issued - kStages); k < issued; ++k) mbar_wait(&full[k % kStages], (uint32_t)(k / kStages) & 1u);
+      for (int k = issued; k < pre_k; ++k)   // requested early, never completed by an arrival
+        if (lane == 0) mbar_arrive(&full[k % kStages]);
+      const int hi = max(issued, pre_k);
+      for (int k = max(0, hi - kStages); k < hi; ++k) mbar_wait(&full[k % kStages], (uint32_t)(k / kStages) & 1u);
     }
   } else if (n_my > 0 && warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -791,13 +821,14 @@ bool score_tc_supported(const KvView& kv, int n_q_heads, const float* qpred) {
 }
 
 cudaError_t launch_score_tc(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s,
-                            int32_t* hist) {
+                            int32_t* hist, bool early) {
   TcParams p;
   p.qpred = qpred;
   p.qraw = nullptr;
   p.qraw_f32 = 0;
   p.len_div = 1;
   p.len_cap = kv.t_max;
+  p.early = early ? 1 : 0;
   p.n_q_heads = n_q_heads;
   p.G = n_q_heads / kv.n_kv;
   p.batch = kv.batch;
@@ -854,6 +885,7 @@ cudaError_t launch_quest_score_tc(const void* q, int q_f32, int n_q_heads, const
   p.qraw_f32 = q_f32;
   p.len_div = quest_page;
   p.len_cap = kv.t_max;
+  p.early = 0;
   p.n_q_heads = n_q_heads;
   p.G = n_q_heads / kv.n_kv;
   p.batch = kv.batch;

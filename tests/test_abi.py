@@ -142,9 +142,16 @@ def test_attend_workspace_rules(lib):
 
 
 def test_decode_workspace_holds_the_partials_and_the_histogram(lib):
-    att = lib.asp_attend_workspace_bytes(8, 32, 8, 128, 2048, 0)
-    dec = lib.asp_decode_workspace_bytes(8, 32, 8, 128, 2048, 0)
-    assert dec >= ((att + 255) // 256) * 256 + 8 * 8 * 2048 * 4
+    # the decode step's attention is planned for one CTA per SM (148 SMs): 64 units
+    # -> 2 splits of 1024 rows; partials (fp32 out + (max, sum) per head and split),
+    # each 256-byte aligned, then the [64, 2048] int32 histogram
+    B, Hq, Hkv, d, C = 8, 32, 8, 128, 2048
+    splits = 148 // (B * Hkv)
+    parts = -(-(B * Hq * splits * d * 4) // 256) * 256 + -(-(B * Hq * splits * 2 * 4) // 256) * 256
+    dec = lib.asp_decode_workspace_bytes(B, Hq, Hkv, d, C, 0)
+    assert dec == parts + B * Hkv * 2048 * 4
+    # fewer splits than the stand-alone attention's plan (3 CTAs per SM)
+    assert dec < lib.asp_attend_workspace_bytes(B, Hq, Hkv, d, C, 0) + B * Hkv * 2048 * 4
     assert lib.asp_decode_workspace_bytes(8, 32, 8, 96, 2048, 0) == 0
     assert lib.asp_decode_workspace_bytes(8, 32, 8, 128, 0, 0) == 0
 
