@@ -359,7 +359,10 @@ def main():
     s_main = st.s_main
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     acct = step_bytes(wl, lens)
-    splits = asp.attend_workspace_bytes(B, Hq, Hkv, d, C, tail) > 0
+    # the decode step's attention has a merge launch when its plan splits the rows:
+    # its workspace then holds partials before the histogram
+    dec_ws = int(asp.lib().asp_decode_workspace_bytes(B, Hq, Hkv, d, C, tail))
+    splits = dec_ws > B * Hkv * 2048 * 4
 
     def one_step(k=None, e2e=False):
         with torch.cuda.stream(s_main):
