@@ -41,7 +41,8 @@ def parse():
     ap.add_argument("--workload", default="qwen3_8b_shaped_32k")
     ap.add_argument("--impl", default="asp", choices=["asp", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-compare", action="store_true", help="skip the page-level and full-attention timings")
+    ap.add_argument("--no-compare", action="store_true",
+                    help="skip the page-level and full-attention timings and the selection recall")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
 
@@ -318,6 +319,33 @@ def comparison_paths(wl, kvd, kv, q_dev, stream, flush, steps):
     return res
 
 
+# ----------------------------------------------------------------------------- selection recall
+def recall_analysis(wl, kv, dev):
+    """Recall of the true next query's top-C set (untimed): the step's own
+    selection (predicted query), the same step with raw ridge coefficients, and
+    the current query reused one step late."""
+    import torch
+    import query_predicted_token_b200 as asp
+    import synth
+    from query_predicted_token_b200.recall import recall_report
+    qhist, q_next = synth.query_history(wl, steps=2)
+    q_t = q_next[0].to(wl.torch_dtype()).to(dev)
+    q_true = q_next[1].to(wl.torch_dtype()).to(dev)     # the model's next query, as attention sees it
+    B, Hq, d, C = wl.batch, wl.n_q_heads, wl.head_dim, wl.C
+    chosen = {}
+    for name, coef in (("predicted", "softmax"), ("predicted_raw_coefficients", "raw")):
+        st = asp.DecodeState(kv, Hq, asp.PredCfg(wl.W, wl.windows, wl.lam, coef), C, qhist.to(dev).contiguous())
+        out = torch.empty(B, Hq, d, dtype=wl.torch_dtype(), device=dev)
+        st.step(q_t, out)
+        torch.cuda.synchronize()
+        chosen[name] = tuple(t.clone() for t in st.selection)
+    res = recall_report(kv, C, q_true, {"current_query": q_t}, chosen)
+    res = {k: round(v, 4) for k, v in res.items()}
+    res["note"] = ("mean over (sequence, KV head) of |S & S_true| / |S_true|, S_true = top C with the true "
+                   "next query; synthetic AR(1) queries (rho %.2f), so an analogue, not the pages' numbers" % wl.rho)
+    return res
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def main():
     args = parse()
@@ -413,6 +441,7 @@ def main():
     e2e_ms = [a.elapsed_time(b) for a, b in ev]
     # the pages' two baselines on the same cache and query: page-level selection, full attention
     compare = None if args.no_compare else comparison_paths(wl, kvd, kv, q_t, s_main, flush, args.steps)
+    recall = None if args.no_compare else recall_analysis(wl, kv, dev)
 
     t_rank, t_e2e = group.slowest(sum(step_ms) / 1e3, sum(e2e_ms) / 1e3)
     (total_bytes,) = group.total(acct["total"] * args.steps)   # ragged batches differ per rank
@@ -454,6 +483,7 @@ def main():
             "gpu_launches": args.steps * (4 + (1 if splits else 0)),
             "cpu_baseline": cpu,
             "comparison": compare,
+            "selection_recall": recall,
         }
         print(json.dumps(line), flush=True)
     group.close()
