@@ -48,7 +48,7 @@
 extern "C" {
 #endif
 
-#define ASP_ABI_VERSION 1
+#define ASP_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define ASP_API __attribute__((visibility("default")))
@@ -235,6 +235,25 @@ ASP_API asp_status asp_sparse_attend_noalloc(const void* q, asp_dtype q_dtype, i
                                              asp_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * The new token's K and V appended to the cache (the cache management that
+ * surrounds the steps; reproduction card, "Key finding", and abstract,
+ * component (2): the cache side keeps the KV cache current while decoding).
+ * k_new, v_new : device [batch, n_kv_heads, head_dim] in kv_dtype, 16-byte aligned.
+ * For every sequence b the token goes to position T = seq_lens[b] (contiguous:
+ * row T of [b, h]; paged: row T % page_size of page page_table[b][T / page_size],
+ * which the caller has allocated), then tail_begin_out[b] = T (when not NULL: the
+ * start of the tail that the next attention covers in full) and seq_lens[b] = T + 1.
+ * kv->seq_lens is read and written on the device and must not be NULL.
+ * quest_meta : NULL, or page bounds as in asp_quest_build_meta (pages of
+ *              quest_page tokens) that are kept current: a token that opens a page
+ *              sets the page's bounds, later tokens widen them.
+ * A sequence at capacity (T == t_max, or past its pages) or whose page is not
+ * valid is left unchanged and ASP_DEV_BAD_PAGE is recorded (asp_device_status).
+ * Asynchronous on `stream`. */
+ASP_API asp_status asp_append_kv(const asp_kv* kv, const void* k_new, const void* v_new, int32_t* tail_begin_out,
+                                 void* quest_meta, int quest_page, asp_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * One asynchronous decode step (steps 1-4).
  * Source: abstract, component (2) (KV selection decoupled from the decoding loop
  * and overlapped with the forward computation).  On one GPU the two ranks of the
@@ -277,6 +296,14 @@ typedef struct {
   asp_event_t ev_fork;
   asp_event_t ev_sel_done;
   asp_event_t* timing;          /* NULL or asp_event_t[8] */
+  /* Optional: the step first appends the new token (asp_append_kv) on s_main, so
+   * that this step's attention, scan and selection all see it.  With k_new set,
+   * kv->seq_lens is advanced on the device and tail_begin (which must then be set,
+   * with max_tail >= 1) is overwritten with the lengths before the append. */
+  const void* k_new;            /* [batch, n_kv_heads, head_dim] kv dtype, or NULL */
+  const void* v_new;
+  void* quest_meta;             /* NULL, or page bounds kept current (see asp_append_kv) */
+  int quest_page;
 } asp_decode_args;
 
 ASP_API asp_status asp_decode_step(const asp_decode_args* args);

@@ -11,6 +11,7 @@ from ._lib import (  # noqa: F401
     ASP_DEV_TAIL_LIMIT,
     ASP_DEV_WAIT_LIMIT,
     AspError,
+    append_kv,
     DecodeState,
     KV,
     PredCfg,

@@ -39,7 +39,8 @@ class AspDecodeArgs(ctypes.Structure):
                 ("qpred", c_void_p), ("scores", c_void_p), ("idx_next", c_void_p), ("count_next", c_void_p),
                 ("out", c_void_p), ("lse", c_void_p), ("workspace", c_void_p), ("workspace_bytes", c_size_t),
                 ("s_main", c_void_p), ("s_side", c_void_p), ("ev_fork", c_void_p), ("ev_sel_done", c_void_p),
-                ("timing", POINTER(c_void_p))]
+                ("timing", POINTER(c_void_p)), ("k_new", c_void_p), ("v_new", c_void_p), ("quest_meta", c_void_p),
+                ("quest_page", c_int)]
 
 
 SIGNATURES = {
@@ -54,6 +55,7 @@ SIGNATURES = {
     "asp_sparse_attend_noalloc": (c_int, [c_void_p, c_int, c_int, POINTER(AspKv), c_void_p, c_void_p, c_int, c_void_p,
                                           c_int, c_void_p, c_void_p, c_void_p]),
     "asp_decode_step": (c_int, [POINTER(AspDecodeArgs)]),
+    "asp_append_kv": (c_int, [POINTER(AspKv), c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p]),
     "asp_wait_selection": (c_int, [c_void_p, c_long]),
     "asp_quest_build_meta": (c_int, [POINTER(AspKv), c_int, c_void_p, c_void_p]),
     "asp_quest_select": (c_int, [c_void_p, c_int, c_int, POINTER(AspKv), c_void_p, c_int, c_int, c_void_p, c_void_p,
@@ -214,6 +216,15 @@ def quest_select(q: torch.Tensor, kv: KV, meta: torch.Tensor, quest_page: int, C
                                                       _ptr(count), _stream(stream)))
 
 
+def append_kv(kv: KV, k_new: torch.Tensor, v_new: torch.Tensor, tail_begin: Optional[torch.Tensor] = None,
+              quest_meta: Optional[torch.Tensor] = None, quest_page: int = 16, stream=None) -> None:
+    """Appends one token per sequence (``k_new, v_new [B, Hkv, d]``) at position
+    ``seq_lens[b]`` and advances ``kv.seq_lens`` on the device; ``tail_begin`` gets the
+    old lengths; ``quest_meta`` (page bounds) is kept current."""
+    _check("asp_append_kv", lib().asp_append_kv(kv.ref, _ptr(k_new), _ptr(v_new), _ptr(tail_begin),
+                                                _ptr(quest_meta), int(quest_page), _stream(stream)))
+
+
 def device_status(stream=None) -> int:
     """Returns (and clears) the device status bits; 0 when no kernel recorded a fault."""
     bits = c_int32(0)
@@ -312,13 +323,21 @@ class DecodeState:
         self.idx[self.cur].copy_(idx)
         self.count[self.cur].copy_(count)
 
-    def step(self, q_t: torch.Tensor, out: torch.Tensor, lse: Optional[torch.Tensor] = None) -> None:
+    def step(self, q_t: torch.Tensor, out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+             k_new: Optional[torch.Tensor] = None, v_new: Optional[torch.Tensor] = None,
+             quest_meta: Optional[torch.Tensor] = None, quest_page: int = 16) -> None:
+        """One decode step; with ``k_new``/``v_new`` the new token is appended first
+        (``kv.seq_lens`` and ``tail_begin`` are then updated on the device)."""
         a = self._args[self.cur]
         a.q_t = q_t.data_ptr()
         a.q_dtype = dtype_code(q_t)
         a.out = out.data_ptr()
         a.lse = lse.data_ptr() if lse is not None else None
         a.ring_start = self.ring_start
+        a.k_new = _ptr(k_new)
+        a.v_new = _ptr(v_new)
+        a.quest_meta = _ptr(quest_meta)
+        a.quest_page = int(quest_page)
         _check("asp_decode_step", self._fn(ctypes.byref(a)))
         self.cur = 1 - self.cur
         self.ring_start = (self.ring_start + 1) % (self.cfg.W + 1)

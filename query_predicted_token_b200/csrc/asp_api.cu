@@ -178,6 +178,19 @@ asp_status check_attend(const void* q, asp_dtype q_dtype, int n_q_heads, const a
   return ASP_OK;
 }
 
+asp_status check_append(const asp_kv* kv, const void* k_new, const void* v_new, const void* meta, int quest_page) {
+  asp_status st = check_kv(kv, true);
+  if (st != ASP_OK) return st;
+  if (!k_new || !v_new || !kv->seq_lens) return ASP_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new)) return ASP_ERR_INVALID_ARG;
+  if (meta) {
+    if (quest_page <= 0 || !aligned16(meta)) return ASP_ERR_INVALID_ARG;
+    if (quest_page % 16 || quest_page > 256) return ASP_ERR_UNSUPPORTED;
+    if (kv->page_size && kv->page_size != quest_page) return ASP_ERR_UNSUPPORTED;
+  }
+  return ASP_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -298,6 +311,11 @@ asp_status asp_decode_step(const asp_decode_args* a) {
   st = check_pred(a->pred, a->ring_start);
   if (st != ASP_OK) return st;
   if (!asp::select_supported(a->kv->t_max, 1) || a->kv->batch > kMaxScoreBatch) return ASP_ERR_UNSUPPORTED;
+  if (a->k_new) {   // the step appends the new token first: it writes seq_lens and tail_begin
+    st = check_append(a->kv, a->k_new, a->v_new, a->quest_meta, a->quest_page);
+    if (st != ASP_OK) return st;
+    if (!a->tail_begin || a->max_tail < 1) return ASP_ERR_INVALID_ARG;
+  }
 
   cudaStream_t sm = reinterpret_cast<cudaStream_t>(a->s_main);
   cudaStream_t ss = reinterpret_cast<cudaStream_t>(a->s_side);
@@ -310,6 +328,9 @@ asp_status asp_decode_step(const asp_decode_args* a) {
   const int B = a->kv->batch;
 
   cudaError_t e = cudaStreamWaitEvent(sm, done, 0);   // idx_cur: the previous step's selection
+  if (e == cudaSuccess && a->k_new)   // before the fork: both streams see the new token
+    e = asp::launch_append(kv, a->k_new, a->v_new, const_cast<int32_t*>(a->kv->seq_lens),
+                           const_cast<int32_t*>(a->tail_begin), a->quest_meta, a->quest_page, sm);
   if (e == cudaSuccess) e = cudaEventRecord(fork, sm);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(ss, fork, 0);
   // side stream: selection for the next step
@@ -368,6 +389,14 @@ asp_status asp_wait_selection(asp_event_t ev_sel_done, long timeout_us) {
   }
 }
 
+asp_status asp_append_kv(const asp_kv* kv, const void* k_new, const void* v_new, int32_t* tail_begin_out,
+                         void* quest_meta, int quest_page, asp_stream_t stream) {
+  asp_status st = check_append(kv, k_new, v_new, quest_meta, quest_page);
+  if (st != ASP_OK) return st;
+  return cuda_status(asp::launch_append(view_of(kv), k_new, v_new, const_cast<int32_t*>(kv->seq_lens), tail_begin_out,
+                                        quest_meta, quest_page, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 asp_status asp_quest_build_meta(const asp_kv* kv, int quest_page, void* meta, asp_stream_t stream) {
   asp_status st = check_kv(kv, false);
   if (st != ASP_OK) return st;
@@ -418,6 +447,7 @@ asp_status asp_device_status(asp_stream_t stream, int32_t* bits_out) {
   if (e == cudaSuccess) e = asp::read_status_attend(s, &v);
   if (e == cudaSuccess) e = asp::read_status_quest(s, &v);
   if (e == cudaSuccess) e = asp::read_status_score_tc(s, &v);
+  if (e == cudaSuccess) e = asp::read_status_append(s, &v);
   if (bits_out) *bits_out = v;
   if (e != cudaSuccess) return ASP_ERR_CUDA;
   return v ? ASP_ERR_DEVICE : ASP_OK;

@@ -44,6 +44,7 @@ cudaError_t read_status_select(cudaStream_t s, int* bits);
 cudaError_t read_status_attend(cudaStream_t s, int* bits);
 cudaError_t read_status_quest(cudaStream_t s, int* bits);
 cudaError_t read_status_score_tc(cudaStream_t s, int* bits);
+cudaError_t read_status_append(cudaStream_t s, int* bits);
 
 // ---- step 1 -----------------------------------------------------------------
 struct PredictArgs {
@@ -76,6 +77,12 @@ struct KvView {
   const int32_t* page_table;
   const int32_t* seq_lens;   // may be null (all t_max)
 };
+// The new token's K and V [batch, n_kv, head_dim] at position seq_lens[b]; then
+// tail_begin[b] (optional) = the old length and seq_lens[b] += 1.  meta: optional
+// page bounds [batch, n_kv, ceil(t_max / quest_page), 2, head_dim] kept current.
+cudaError_t launch_append(const KvView& kv, const void* k_new, const void* v_new, int32_t* seq_lens,
+                          int32_t* tail_begin, void* meta, int quest_page, cudaStream_t s);
+
 // hist: optional [batch * n_kv, 2048] int32 counts of the scores' top 11 key bits
 // (must be zero on entry); the selection then skips its own first pass.
 // early: the previous kernel of the stream writes only qpred (and clears hist), and

@@ -59,12 +59,15 @@ int main(void) {
   printf("asp_kv %zu %zu %zu %zu %zu\n", sizeof(asp_kv), offsetof(asp_kv, k), offsetof(asp_kv, page_size),
          offsetof(asp_kv, page_table), offsetof(asp_kv, seq_lens));
   printf("asp_pred_cfg %zu %zu %zu\n", sizeof(asp_pred_cfg), offsetof(asp_pred_cfg, windows), offsetof(asp_pred_cfg, lambda));
-  printf("asp_decode_args %zu %zu %zu %zu %zu\n", sizeof(asp_decode_args), offsetof(asp_decode_args, kv),
-         offsetof(asp_decode_args, workspace_bytes), offsetof(asp_decode_args, s_main), offsetof(asp_decode_args, timing));
+  printf("asp_decode_args %zu %zu %zu %zu %zu %zu %zu\n", sizeof(asp_decode_args), offsetof(asp_decode_args, kv),
+         offsetof(asp_decode_args, workspace_bytes), offsetof(asp_decode_args, s_main), offsetof(asp_decode_args, timing),
+         offsetof(asp_decode_args, k_new), offsetof(asp_decode_args, quest_page));
   return 0;
 }
 '''
-    with tempfile.TemporaryDirectory() as d:
+    scratch = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "_build")
+    os.makedirs(scratch, exist_ok=True)
+    with tempfile.TemporaryDirectory(dir=scratch) as d:
         c = os.path.join(d, "l.c")
         open(c, "w").write(src)
         exe = os.path.join(d, "l")
@@ -74,11 +77,11 @@ int main(void) {
     assert lines["asp_kv"] == [ctypes.sizeof(K), K.k.offset, K.page_size.offset, K.page_table.offset, K.seq_lens.offset]
     assert lines["asp_pred_cfg"] == [ctypes.sizeof(P), P.windows.offset, P.lam.offset]
     assert lines["asp_decode_args"] == [ctypes.sizeof(D), D.kv.offset, D.workspace_bytes.offset, D.s_main.offset,
-                                        D.timing.offset]
+                                        D.timing.offset, D.k_new.offset, D.quest_page.offset]
 
 
 def test_version_and_status_strings(lib):
-    assert lib.asp_abi_version() == 1
+    assert lib.asp_abi_version() == 2
     assert L.status_string(L.ASP_OK) == "ok"
     assert "workspace" in L.status_string(L.ASP_ERR_WORKSPACE)
     assert L.status_string(99) == "unknown status"
@@ -113,6 +116,22 @@ def test_score_rejects_bad_groups(lib):
     assert lib.asp_score_keys(FAKE, 5, ctypes.byref(kv), FAKE, None) == L.ASP_ERR_INVALID_ARG   # 5 % 2
     assert lib.asp_score_keys(None, 8, ctypes.byref(kv), FAKE, None) == L.ASP_ERR_INVALID_ARG
     assert lib.asp_score_keys(FAKE, 8, None, FAKE, None) == L.ASP_ERR_INVALID_ARG
+
+
+def test_append_validation(lib):
+    """asp_append_kv checks everything on the host; nothing here reaches a kernel."""
+    kv = _kv(seq_lens=FAKE)
+    call = lambda kv, k=FAKE, v=FAKE, meta=None, page=16: lib.asp_append_kv(ctypes.byref(kv), k, v, None, meta, page, None)
+    assert call(_kv()) == L.ASP_ERR_INVALID_ARG                     # lengths must live on the device
+    assert call(kv, k=None) == L.ASP_ERR_INVALID_ARG
+    assert call(kv, v=None) == L.ASP_ERR_INVALID_ARG
+    assert call(_kv(seq_lens=FAKE, v=None)) == L.ASP_ERR_INVALID_ARG  # the cache needs its values
+    assert call(kv, k=FAKE + 4) == L.ASP_ERR_INVALID_ARG              # not 16-byte aligned
+    assert call(kv, meta=FAKE, page=0) == L.ASP_ERR_INVALID_ARG
+    assert call(kv, meta=FAKE, page=24) == L.ASP_ERR_UNSUPPORTED
+    paged = _kv(seq_lens=FAKE, page_size=16, page_table=FAKE, max_pages=64, n_pages=200)
+    assert call(paged, meta=FAKE, page=32) == L.ASP_ERR_UNSUPPORTED  # bounds pages must be the cache's pages
+    assert call(_kv(seq_lens=FAKE, head_dim=96)) == L.ASP_ERR_UNSUPPORTED
 
 
 def test_select_validation(lib):

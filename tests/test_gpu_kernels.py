@@ -141,6 +141,65 @@ def test_decode_step_on_whole_pages_selects_the_top_scores():
             assert_scores_close(scores[b, h, :lens[b]], ref, pred[b, h * G:(h + 1) * G], keys[b][h], f"b{b}h{h}")
 
 
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.bfloat16, 64), (torch.float32, 128)])
+@pytest.mark.parametrize("page_size", [0, 16])
+def test_append_kv_writes_the_token_and_keeps_the_page_bounds(dtype, d, page_size):
+    B, Hkv, P = 3, 2, 16
+    if page_size == 0:
+        lens = [40, 95, 17]
+        kvd, kv = make_cache(B, Hkv, d, 96, dtype, lens, 0, seed=d)
+    else:   # every sequence owns 4 pages (64 tokens) and uses fewer: the append has room
+        lens = [40, 63, 17]
+        kvd, _ = make_cache(B, Hkv, d, 64, dtype, [64] * B, 16, seed=d + 1)
+        kvd["seq_lens"] = torch.tensor(lens, dtype=torch.int32, device=DEV)
+        kv = asp.KV(kvd["k"], kvd["v"], kvd["seq_lens"], kvd["page_table"], t_max=64)
+    npm = (kv.t_max + P - 1) // P
+    meta = torch.zeros(B, Hkv, npm, 2, d, dtype=dtype, device=DEV)
+    asp.quest_build_meta(kv, P, meta)
+    k0, v0 = kvd["k"].clone(), kvd["v"].clone()
+    g = _gen(21)
+    k_new = torch.randn(B, Hkv, d, generator=g).to(dtype).to(DEV)
+    v_new = torch.randn(B, Hkv, d, generator=g).to(dtype).to(DEV)
+    tail = torch.full((B,), -7, dtype=torch.int32, device=DEV)
+    asp.append_kv(kv, k_new, v_new, tail, meta, P)
+    torch.cuda.synchronize()
+    assert kvd["seq_lens"].cpu().tolist() == [t + 1 for t in lens]
+    assert tail.cpu().tolist() == lens
+    for b in range(B):
+        T_b = lens[b]
+        for h in range(Hkv):
+            if page_size == 0:
+                at = (b, h, T_b)
+            else:
+                at = (int(kvd["page_table"][b, T_b // P]), h, T_b % P)
+            assert torch.equal(kvd["k"][at], k_new[b, h]) and torch.equal(kvd["v"][at], v_new[b, h])
+            kvd["k"][at], kvd["v"][at] = k0[at], v0[at]   # everything else is untouched
+    assert torch.equal(kvd["k"], k0) and torch.equal(kvd["v"], v0)
+    # the kept bounds equal bounds rebuilt from the cache with the token in it
+    kvd["k"].copy_(k0)
+    for b in range(B):
+        for h in range(Hkv):
+            at = (b, h, lens[b]) if page_size == 0 else (int(kvd["page_table"][b, lens[b] // P]), h, lens[b] % P)
+            kvd["k"][at] = k_new[b, h]
+    ref = torch.zeros_like(meta)
+    asp.quest_build_meta(kv, P, ref)
+    torch.cuda.synchronize()
+    for b in range(B):
+        n = (lens[b] + 1 + P - 1) // P
+        assert torch.equal(meta[b, :, :n], ref[b, :, :n])
+
+
+def test_append_kv_at_capacity_changes_nothing_and_reports_it():
+    kvd, kv = make_cache(2, 2, 64, 32, torch.bfloat16, [32, 5])
+    k_new = torch.ones(2, 2, 64, dtype=torch.bfloat16, device=DEV)
+    before = kvd["k"].clone()
+    asp.append_kv(kv, k_new, k_new)
+    torch.cuda.synchronize()
+    assert kvd["seq_lens"].cpu().tolist() == [32, 6]          # the full sequence keeps its length
+    assert torch.equal(kvd["k"][0], before[0])
+    assert asp.device_status() & asp.ASP_DEV_BAD_PAGE          # reported (and cleared)
+
+
 def test_score_empty_sequence_writes_nothing():
     kvd, kv = make_cache(2, 2, 128, 64, torch.bfloat16, [0, 40])
     qpred = torch.randn(2, 8, 128, generator=_gen(1)).to(DEV)

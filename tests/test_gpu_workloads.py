@@ -216,3 +216,60 @@ def test_decode_selection_when_most_tokens_survive_the_first_digit():
     for b in range(B):
         for h in range(Hkv):
             assert_valid_topk(scores[b, h], int(lens[b]), C, idx[b, h], int(cnt[b, h]), f"b{b}h{h}")
+
+
+@pytest.mark.parametrize("page_size", [0, 16])
+def test_decode_steps_that_append_the_new_token(page_size):
+    """Three decode steps, each appending the new token first: the lengths advance,
+    the attention covers the previous selection plus the new token (its tail), the
+    next selection is the top C of the step's own scores over every token so far,
+    and the kept page bounds equal bounds rebuilt from the grown cache."""
+    from test_gpu_kernels import make_cache
+    B, Hkv, G, d, C, W, P, cap = 2, 8, 4, 128, 128, 8, 16, 1024
+    lens0 = [1000, 700]
+    if page_size == 0:
+        kvd, _ = make_cache(B, Hkv, d, cap, torch.bfloat16, lens0, 0, seed=41)
+    else:   # every sequence owns all its pages; the lengths start shorter
+        kvd, _ = make_cache(B, Hkv, d, cap, torch.bfloat16, [cap] * B, P, seed=41)
+        kvd["seq_lens"] = torch.tensor(lens0, dtype=torch.int32, device=DEV)
+    kv = asp.KV(kvd["k"], kvd["v"], kvd["seq_lens"], kvd["page_table"], t_max=cap)
+    meta = torch.zeros(B, Hkv, cap // P, 2, d, dtype=torch.bfloat16, device=DEV)
+    asp.quest_build_meta(kv, P, meta)
+    g = torch.Generator().manual_seed(42)
+    qhist = torch.randn(B, Hkv * G, W + 1, d, generator=g).to(DEV).contiguous()
+    tail = torch.tensor(lens0, dtype=torch.int32, device=DEV)
+    st = asp.DecodeState(kv, Hkv * G, asp.PredCfg(W, (4, 8), 1e-2), C, qhist, max_tail=1, tail_begin=tail)
+    idx0, cnt0 = synth.random_selection(B, Hkv, C, lens0, seed=43)
+    st.set_selection(idx0.to(DEV), cnt0.to(DEV))
+    for step in range(3):
+        q = torch.randn(B, Hkv * G, d, generator=g).to(torch.bfloat16).to(DEV)
+        k_new = torch.randn(B, Hkv, d, generator=g).to(torch.bfloat16).to(DEV)
+        v_new = torch.randn(B, Hkv, d, generator=g).to(torch.bfloat16).to(DEV)
+        old = kvd["seq_lens"].cpu().tolist()
+        idx_cur, cnt_cur = st.idx[st.cur].cpu().numpy(), st.count[st.cur].cpu().numpy()
+        out = torch.empty(B, Hkv * G, d, dtype=torch.bfloat16, device=DEV)
+        lse = torch.empty(B, Hkv * G, device=DEV)
+        st.step(q, out, lse, k_new, v_new, meta, P)
+        assert asp.wait_selection(st.ev_sel_done, 60_000_000) == 0
+        torch.cuda.synchronize()
+        assert asp.device_status() == 0
+        new = kvd["seq_lens"].cpu().tolist()
+        assert new == [t + 1 for t in old] and tail.cpu().tolist() == old
+        keys, vals = host_sequences(kvd)
+        scores = st.scores.cpu().numpy()
+        idx1, cnt1 = (t.cpu().numpy() for t in st.selection)
+        for b in range(B):
+            assert np.array_equal(keys[b][:, old[b]], np64(k_new[b]))      # the token is in the cache
+            for h in range(Hkv):
+                S = oracle.attend.attended_set(idx_cur[b, h], int(cnt_cur[b, h]), old[b], new[b])
+                assert old[b] in S.tolist()
+                ref_o, ref_l = oracle.attend_set(np64(q[b, h * G:(h + 1) * G]), keys[b][h], vals[b][h], S)
+                assert_out_close(out[b, h * G:(h + 1) * G], ref_o, torch.bfloat16, f"step {step} b{b}h{h}")
+                assert_lse_close(lse[b, h * G:(h + 1) * G], ref_l)
+                assert_valid_topk(scores[b, h], new[b], C, idx1[b, h], int(cnt1[b, h]), f"step {step} b{b}h{h}")
+    ref = torch.zeros_like(meta)
+    asp.quest_build_meta(kv, P, ref)
+    torch.cuda.synchronize()
+    for b in range(B):
+        n = -(-int(kvd["seq_lens"][b]) // P)
+        assert torch.equal(meta[b, :, :n], ref[b, :, :n])
