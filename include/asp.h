@@ -267,7 +267,10 @@ ASP_API asp_status asp_append_kv(const asp_kv* kv, const void* k_new, const void
  * priority than s_main, so that its kernels get SMs before the attention's.
  * The caller swaps idx_cur/idx_next (and count_*) between steps, advances
  * ring_start by one, and must not reuse q_t, qpred, scores or idx_next before
- * ev_sel_done completes.  workspace: at least asp_decode_workspace_bytes(...)
+ * ev_sel_done completes.  While s_main is being captured (CUDA graphs) the step
+ * leaves out its wait for ev_sel_done: the caller then orders the graph launches on
+ * one stream, and ends each capture with s_main waiting for ev_sel_done, so that
+ * the graph joins both streams.  workspace: at least asp_decode_workspace_bytes(...)
  * bytes, 256-byte aligned, no initialisation needed (ASP_ERR_WORKSPACE otherwise).  timing: NULL, or 8 events recorded around the kernels
  * (begin/end of predict, score, select on s_side; attend on s_main) for profiling. */
 typedef struct {
@@ -307,6 +310,17 @@ typedef struct {
 } asp_decode_args;
 
 ASP_API asp_status asp_decode_step(const asp_decode_args* args);
+
+/* CUDA graphs of decode steps (no counterpart in the pages: launch plumbing).
+ * graph: a cudaGraph_t captured from asp_decode_step calls (see above).  The graph
+ * is instantiated so that each kernel keeps the priority of the stream it was
+ * captured from: the selection chain then stays ahead of the attention, as in
+ * eager steps (a plain instantiation runs every node at the launch stream's
+ * priority).  The caller keeps the graph alive while it uses the instantiation,
+ * and frees the instantiation with asp_graph_destroy. */
+ASP_API asp_status asp_graph_instantiate(void* graph, void** exec_out);
+ASP_API asp_status asp_graph_launch(void* exec, asp_stream_t stream);
+ASP_API asp_status asp_graph_destroy(void* exec);
 
 /* Host wait for a selection with a time limit (polls the event; never blocks past
  * timeout_us).  Returns ASP_OK, ASP_ERR_TIMEOUT or ASP_ERR_CUDA. */

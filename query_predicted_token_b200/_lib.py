@@ -56,6 +56,9 @@ SIGNATURES = {
                                           c_int, c_void_p, c_void_p, c_void_p]),
     "asp_decode_step": (c_int, [POINTER(AspDecodeArgs)]),
     "asp_append_kv": (c_int, [POINTER(AspKv), c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p]),
+    "asp_graph_instantiate": (c_int, [c_void_p, POINTER(c_void_p)]),
+    "asp_graph_launch": (c_int, [c_void_p, c_void_p]),
+    "asp_graph_destroy": (c_int, [c_void_p]),
     "asp_wait_selection": (c_int, [c_void_p, c_long]),
     "asp_quest_build_meta": (c_int, [POINTER(AspKv), c_int, c_void_p, c_void_p]),
     "asp_quest_select": (c_int, [c_void_p, c_int, c_int, POINTER(AspKv), c_void_p, c_int, c_int, c_void_p, c_void_p,
@@ -339,6 +342,61 @@ class DecodeState:
         a.quest_meta = _ptr(quest_meta)
         a.quest_page = int(quest_page)
         _check("asp_decode_step", self._fn(ctypes.byref(a)))
+        self.cur = 1 - self.cur
+        self.ring_start = (self.ring_start + 1) % (self.cfg.W + 1)
+
+    # ---- CUDA graphs -------------------------------------------------------
+    def capture(self, q_t: torch.Tensor, out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                k_new: Optional[torch.Tensor] = None, v_new: Optional[torch.Tensor] = None,
+                quest_meta: Optional[torch.Tensor] = None, quest_page: int = 16) -> int:
+        """Captures one CUDA graph per state of the step cycle (selection parity x
+        ring position: lcm(2, W + 1) graphs), starting from the current state, each
+        one :meth:`step` on these fixed buffers (write each step's query, and K/V when
+        appending, into them before :meth:`replay`).  Run one eager :meth:`step` first
+        (the library prepares its kernels on first use).  Returns the cycle length."""
+        import math
+        n = 2 * (self.cfg.W + 1) // math.gcd(2, self.cfg.W + 1)
+        cur0, ring0 = self.cur, self.ring_start
+        main0 = self.s_main
+        timing_on = bool(self._args[0].timing)
+        cap = torch.cuda.Stream(device=self.kv.k.device)
+        self.graphs = []
+        try:
+            self.s_main = cap
+            self._args = [self._build_args(0), self._build_args(1)]
+            for a in self._args:   # no timing events inside a graph
+                a.timing = None
+            for _ in range(n):
+                g = torch.cuda.CUDAGraph(keep_graph=True)
+                with torch.cuda.graph(g, stream=cap):
+                    self.step(q_t, out, lse, k_new, v_new, quest_meta, quest_page)
+                    cap.wait_event(self.ev_sel_done)   # the graph joins the side stream
+                ex = c_void_p()
+                _check("asp_graph_instantiate", lib().asp_graph_instantiate(c_void_p(g.raw_cuda_graph()),
+                                                                            ctypes.byref(ex)))
+                self.graphs.append((g, ex))
+        finally:
+            self.s_main = main0
+            self._args = [self._build_args(0), self._build_args(1)]
+            self.set_timing(timing_on) if self._timing_arr is not None else None
+            self.cur, self.ring_start = cur0, ring0
+        # the events were last recorded inside the captures: record them once outside
+        self.ev_fork.record(self.s_main)
+        self.ev_sel_done.record(self.s_main)
+        self._graph_at = 0
+        return n
+
+    def release_graphs(self) -> None:
+        for _, ex in getattr(self, "graphs", []):
+            lib().asp_graph_destroy(ex)
+        self.graphs = []
+
+    def replay(self) -> None:
+        """One step by replaying the captured graph of the current state on the
+        current stream (the graphs must have been captured from this state on)."""
+        _check("asp_graph_launch", lib().asp_graph_launch(self.graphs[self._graph_at][1],
+                                                          _stream(torch.cuda.current_stream())))
+        self._graph_at = (self._graph_at + 1) % len(self.graphs)
         self.cur = 1 - self.cur
         self.ring_start = (self.ring_start + 1) % (self.cfg.W + 1)
 

@@ -327,7 +327,12 @@ asp_status asp_decode_step(const asp_decode_args* a) {
   const KvView kv = view_of(a->kv);
   const int B = a->kv->batch;
 
-  cudaError_t e = cudaStreamWaitEvent(sm, done, 0);   // idx_cur: the previous step's selection
+  // idx_cur is the previous step's selection.  While s_main is being captured into
+  // a graph the wait is left out: launches of the captured graph on one stream are
+  // ordered, and each graph ends with both streams joined.
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(sm, &capture);
+  if (e == cudaSuccess && capture == cudaStreamCaptureStatusNone) e = cudaStreamWaitEvent(sm, done, 0);
   if (e == cudaSuccess && a->k_new)   // before the fork: both streams see the new token
     e = asp::launch_append(kv, a->k_new, a->v_new, const_cast<int32_t*>(a->kv->seq_lens),
                            const_cast<int32_t*>(a->tail_begin), a->quest_meta, a->quest_page, sm);
@@ -373,6 +378,26 @@ asp_status asp_decode_step(const asp_decode_args* a) {
                            a->tail_begin, a->max_tail, a->out, a->lse, a->workspace, plan, sm);
   if (e == cudaSuccess) e = mark(7, sm);
   return cuda_status(e);
+}
+
+asp_status asp_graph_instantiate(void* graph, void** exec_out) {
+  if (!graph || !exec_out) return ASP_ERR_INVALID_ARG;
+  cudaGraphExec_t ex = nullptr;
+  const cudaError_t e = cudaGraphInstantiateWithFlags(&ex, static_cast<cudaGraph_t>(graph),
+                                                      cudaGraphInstantiateFlagUseNodePriority);
+  if (e != cudaSuccess) return ASP_ERR_CUDA;
+  *exec_out = ex;
+  return ASP_OK;
+}
+
+asp_status asp_graph_launch(void* exec, asp_stream_t stream) {
+  if (!exec) return ASP_ERR_INVALID_ARG;
+  return cuda_status(cudaGraphLaunch(static_cast<cudaGraphExec_t>(exec), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+asp_status asp_graph_destroy(void* exec) {
+  if (!exec) return ASP_ERR_INVALID_ARG;
+  return cuda_status(cudaGraphExecDestroy(static_cast<cudaGraphExec_t>(exec)));
 }
 
 asp_status asp_wait_selection(asp_event_t ev_sel_done, long timeout_us) {

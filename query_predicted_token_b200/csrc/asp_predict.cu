@@ -305,8 +305,7 @@ cudaError_t launch_t(const PredictArgs& a, cudaStream_t s) {
   const size_t smem = kWarps * kSolveBytes;
   auto kern = predict_kernel<D, NV>;
   if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
-  kern<<<grid, kWarps * 32, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_prio(kern, dim3(grid), dim3(kWarps * 32), smem, s, a);
 }
 
 template <int D>

@@ -273,3 +273,53 @@ def test_decode_steps_that_append_the_new_token(page_size):
     for b in range(B):
         n = -(-int(kvd["seq_lens"][b]) // P)
         assert torch.equal(meta[b, :, :n], ref[b, :, :n])
+
+
+def test_graph_replay_reproduces_eager_steps_bit_for_bit():
+    """Steps replayed from captured CUDA graphs (one per parity x ring state, with
+    the append of the new token) give exactly the eager steps' outputs, selections,
+    lengths and tails."""
+    from test_gpu_kernels import make_cache
+    B, Hkv, G, d, C, W, cap = 2, 8, 4, 128, 128, 4, 2048
+    lens0 = [1500, 900]
+    states = []
+    for _ in range(2):
+        kvd, _ = make_cache(B, Hkv, d, cap, torch.bfloat16, lens0, 0, seed=51)
+        kv = asp.KV(kvd["k"], kvd["v"], kvd["seq_lens"], t_max=cap)
+        qhist = torch.randn(B, Hkv * G, W + 1, d, generator=torch.Generator().manual_seed(52)).to(DEV).contiguous()
+        tail = torch.tensor(lens0, dtype=torch.int32, device=DEV)
+        st = asp.DecodeState(kv, Hkv * G, asp.PredCfg(W, (2, 4), 1e-2), C, qhist, max_tail=1, tail_begin=tail)
+        idx0, cnt0 = synth.random_selection(B, Hkv, C, lens0, seed=53)
+        st.set_selection(idx0.to(DEV), cnt0.to(DEV))
+        bufs = dict(q=torch.empty(B, Hkv * G, d, dtype=torch.bfloat16, device=DEV),
+                    k=torch.empty(B, Hkv, d, dtype=torch.bfloat16, device=DEV),
+                    v=torch.empty(B, Hkv, d, dtype=torch.bfloat16, device=DEV),
+                    out=torch.empty(B, Hkv * G, d, dtype=torch.bfloat16, device=DEV),
+                    lse=torch.empty(B, Hkv * G, device=DEV))
+        states.append((kvd, st, tail, bufs))
+    g = torch.Generator().manual_seed(54)
+    inputs = [(torch.randn(B, Hkv * G, d, generator=g), torch.randn(B, Hkv, d, generator=g),
+               torch.randn(B, Hkv, d, generator=g)) for _ in range(14)]
+    graphed = False
+    for step, (q, k, v) in enumerate(inputs):
+        for i, (kvd, st, tail, bf) in enumerate(states):
+            bf["q"].copy_(q.to(torch.bfloat16))
+            bf["k"].copy_(k.to(torch.bfloat16))
+            bf["v"].copy_(v.to(torch.bfloat16))
+            if i == 1 and step >= 1:
+                if not graphed:   # after one eager step: one graph per state of the cycle
+                    assert st.capture(bf["q"], bf["out"], bf["lse"], bf["k"], bf["v"]) == 10   # lcm(2, W + 1)
+                    graphed = True
+                st.replay()
+            else:
+                st.step(bf["q"], bf["out"], bf["lse"], bf["k"], bf["v"])
+            torch.cuda.current_stream().wait_event(st.ev_sel_done)
+        torch.cuda.synchronize()
+        (ka, sa, ta, ba), (kb, sb, tb, bb) = states
+        assert torch.equal(ba["out"], bb["out"]) and torch.equal(ba["lse"], bb["lse"]), f"step {step}"
+        for x, y in zip(sa.selection, sb.selection):
+            assert torch.equal(x, y), f"step {step}"
+        assert torch.equal(ka["seq_lens"], kb["seq_lens"]) and torch.equal(ta, tb)
+    assert states[1][1].ring_start == states[0][1].ring_start and states[1][1].cur == states[0][1].cur
+    states[1][1].release_graphs()
+    assert asp.device_status() == 0
