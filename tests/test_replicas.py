@@ -60,8 +60,12 @@ def _rank_dies(rank: int, world: int, port: int, q) -> None:
     """Rank 1 exits abruptly after joining (no teardown, so its sockets close at
     once); rank 0 then enters a collective."""
     _rank_env(rank, world, port)
-    g = ReplicaGroup("gloo", "cpu", timeout_s=5)
-    g.barrier()   # both ranks fully connected before one of them leaves
+    try:   # a loaded host can take seconds to connect: report a failure instead of going silent
+        g = ReplicaGroup("gloo", "cpu", timeout_s=30)
+        g.barrier()   # both ranks fully connected before one of them leaves
+    except Exception as e:
+        q.put((rank, "setup failed", repr(e)))
+        os._exit(1)
     if rank == 1:
         q.put((rank, "raised", None))
         q.close()
@@ -141,6 +145,8 @@ def test_two_gloo_ranks_aggregate():
 
 
 def test_dead_rank_ends_collective_with_error():
+    # the survivor's collective fails when the dead rank's sockets close, well inside
+    # the group's 30 s timeout
     res = _run(_rank_dies, join_s=90.0)
     assert res[1][1] == "raised"
     assert res[0][1] == "error", res[0]
