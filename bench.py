@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--no-compare", action="store_true",
                     help="skip the page-level and full-attention timings and the selection recall")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--layers", type=int, default=1,
+                    help="also time a stack of this many layers (each with its own cache), steady-state period")
     return ap.parse_args()
 
 
@@ -346,6 +348,70 @@ def recall_analysis(wl, kv, dev):
     return res
 
 
+# ----------------------------------------------------------------------------- multi-layer stack
+def multi_layer_period(wl, layers, tokens, dev):
+    """Steady-state decode period of a stack of `layers` layers, each with its own
+    cache and query history: per token, layer l's attention runs on the main stream
+    in layer order, and every layer's prediction, scan and selection run on one
+    shared side stream (the cache side of the pages' two ranks).  The period is the
+    time of `tokens` tokens over `tokens`, after 2 warm-up tokens; a layer is only
+    allocated while the device keeps 20% more memory free than it needs."""
+    import torch
+    import query_predicted_token_b200 as asp
+    import synth
+    B, Hq, Hkv, d, C = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.C
+    e = 2 if wl.kv_dtype == "bf16" else 4
+    per_layer = 2 * B * Hkv * wl.t_max * d * e
+    main_s = torch.cuda.current_stream()
+    side_s = torch.cuda.Stream(priority=-100)
+    states, outs, qs = [], [], []
+    for l in range(layers):
+        free, _ = torch.cuda.mem_get_info(dev)
+        if free < 1.2 * per_layer + (2 << 30):
+            break
+        wl_l = wl.replace(seed=wl.seed + 1009 * (l + 1))
+        kvd = synth.kv_cache(wl_l, dev)
+        kv = asp.KV(kvd["k"], kvd["v"], kvd["seq_lens"], kvd["page_table"], t_max=wl.t_max)
+        qhist, q_next = synth.query_history(wl_l, steps=1)
+        st = asp.DecodeState(kv, Hq, asp.PredCfg(wl.W, wl.windows, wl.lam), C, qhist.to(dev).contiguous(),
+                             s_main=main_s, s_side=side_s)
+        lens = kvd["seq_lens"].cpu().tolist()
+        idx0, cnt0 = synth.random_selection(B, Hkv, C, lens, seed=wl_l.seed + 99)
+        st.set_selection(idx0.to(dev), cnt0.to(dev))
+        st._kvd = kvd   # keep the cache alive with its state
+        states.append(st)
+        qs.append(q_next[0].to(wl.torch_dtype()).to(dev))
+        outs.append(torch.empty(B, Hq, d, dtype=wl.torch_dtype(), device=dev))
+    n = len(states)
+    if n == 0:
+        return {"layers": 0, "note": "not enough device memory for one layer"}
+
+    def token():
+        for l in range(n):
+            states[l].step(qs[l], outs[l])
+
+    for _ in range(2):
+        token()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(main_s)
+    for _ in range(tokens):
+        token()
+    main_s.wait_event(states[-1].ev_sel_done)   # the last layer's selection ends the window
+    b.record(main_s)
+    torch.cuda.synchronize()
+    period_us = a.elapsed_time(b) * 1e3 / tokens
+    lens = synth.workloads.sequence_lengths(wl).tolist()
+    step_b = step_bytes(wl, lens)["total"]
+    res = {"layers": n, "requested_layers": layers, "tokens": tokens, "period_us": round(period_us, 1),
+           "per_layer_us": round(period_us / n, 2), "gbs": round(step_b * n / (period_us / 1e6) / 1e9, 1),
+           "note": "per token: attention of every layer on the main stream in layer order, prediction, scan and "
+                   "selection of every layer on one side stream; no model weights or other layers' compute"}
+    del states
+    torch.cuda.empty_cache()
+    return res
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def main():
     args = parse()
@@ -442,6 +508,10 @@ def main():
     # the pages' two baselines on the same cache and query: page-level selection, full attention
     compare = None if args.no_compare else comparison_paths(wl, kvd, kv, q_t, s_main, flush, args.steps)
     recall = None if args.no_compare else recall_analysis(wl, kv, dev)
+    stack = multi_layer_period(wl, args.layers, args.steps, dev) if args.layers > 1 else None
+    if stack and compare and stack.get("layers"):
+        for k in ("page_level", "full_attention"):   # one layer's measured step times the layer count
+            stack[k + "_period_us_from_one_layer"] = round(compare[k]["step_us"] * stack["layers"], 1)
 
     t_rank, t_e2e = group.slowest(sum(step_ms) / 1e3, sum(e2e_ms) / 1e3)
     (total_bytes,) = group.total(acct["total"] * args.steps)   # ragged batches differ per rank
@@ -484,6 +554,7 @@ def main():
             "cpu_baseline": cpu,
             "comparison": compare,
             "selection_recall": recall,
+            "multi_layer": stack,
         }
         print(json.dumps(line), flush=True)
     group.close()
