@@ -20,7 +20,7 @@
 //    substitutions in fp64 (the lag Gram's condition number is ~1e3 on AR(1)
 //    histories; fp64 keeps the coefficients' error far below the output bound);
 //  * the Cholesky is warp-parallel (pivot computed by every lane, column
-//    broadcast by shuffles, lane i updates row i).
+//    broadcast through shared memory, lane i updates row i).
 #include "asp_common.cuh"
 #include "asp_internal.h"
 
@@ -149,7 +149,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) predict_kernel(PredictArgs a) 
   const int wm = a.wmax;
   constexpr int WMAX = NV - 1;   // lags the registers can hold
   // Cholesky A = L L^T with lane i holding row i of the lower triangle in
-  // registers; the pivot comes from lane k and column k is broadcast by shuffles.
+  // registers; the pivot comes from lane k by a shuffle, column k through shared
+  // memory.
   {
     double arow[WMAX];
 #pragma unroll
@@ -167,11 +168,17 @@ __global__ void __launch_bounds__(kWarps * 32, 1) predict_kernel(PredictArgs a) 
         } else if (lane > k) {
           arow[k] = lik;
         }
+        // column k goes through shared memory: one store per lane and one broadcast
+        // load per later column, instead of two shuffles per later column
+        double* col = invd + 32;
+        col[lane] = lik;
+        __syncwarp();
 #pragma unroll
         for (int j = k + 1; j < WMAX; ++j) {
-          const double ljk = __shfl_sync(0xffffffffu, lik, j);
+          const double ljk = col[j];
           if (j < wm && lane >= j && lane < wm) arow[j] -= lik * ljk;
         }
+        __syncwarp();   // the next column overwrites col
       }
     }
     if (lane < wm) {
