@@ -28,8 +28,15 @@ namespace asp {
 namespace {
 
 constexpr int kWarps = 4;
-constexpr int kLda = 33;   // row stride (doubles) of the lag Gram: column accesses hit distinct banks
-constexpr size_t kSolveBytes = (32 * kLda + 3 * 32) * 8;   // A[32][33], rhs/beta, 1/diag, spare (fp64)
+// Per-warp solve area for NV history vectors (NV - 1 lags): the lag Gram A with an
+// odd row stride (column accesses hit distinct banks), then rhs/beta, 1/diag and a
+// spare column of 32 doubles each (fp64).
+template <int NV>
+struct Solve {
+  static constexpr int kRows = NV - 1;
+  static constexpr int kLda = (NV - 1) | 1;
+  static constexpr size_t kBytes = ((size_t)kRows * kLda + 3 * 32) * 8;
+};
 
 // 1/sqrt(x) for x > 0 in fp64: the fp32 hardware estimate refined by one
 // Newton-Raphson step y <- y (3 - x y^2) / 2, which squares its relative error
@@ -41,13 +48,14 @@ __device__ __forceinline__ double rsqrt_f64(double x) {
 
 // Stores the reduced pair `q` (lane's pair of a round) into the solve arrays:
 // pairs (i >= 1, j >= 1) are lag-Gram entries, pairs (i >= 1, 0) the right-hand side.
+template <int LDA>
 __device__ __forceinline__ void store_pair(int q, float val, int wmax, double lam, double* A, double* rhs) {
   int qi = (int)((sqrtf(8.f * q + 1.f) - 1.f) * 0.5f);
   while (qi * (qi + 1) / 2 > q) --qi;
   while ((qi + 1) * (qi + 2) / 2 <= q) ++qi;
   const int qj = q - qi * (qi + 1) / 2;
   if (qi >= 1 && qi <= wmax) {
-    if (qj >= 1) A[(qi - 1) * kLda + (qj - 1)] = (double)val + (qi == qj ? lam : 0.0);
+    if (qj >= 1) A[(qi - 1) * LDA + (qj - 1)] = (double)val + (qi == qj ? lam : 0.0);
     else rhs[qi - 1] = (double)val;
   }
 }
@@ -70,7 +78,7 @@ struct GramCol {
       for (int k = P % 32 + 1; k < 32; ++k) part[k] = 0.f;
       ReduceScatter<32, 16>::run(part, lane);
       const int q = (P / 32) * 32 + lane;
-      if (q < NPAIR) store_pair(q, part[0], wmax, lam, A, rhs);
+      if (q < NPAIR) store_pair<Solve<NV>::kLda>(q, part[0], wmax, lam, A, rhs);
     }
     if constexpr (J < I) GramCol<NV, CPL, I, J + 1>::run(h, part, lane, wmax, lam, A, rhs);
   }
@@ -100,8 +108,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) predict_kernel(PredictArgs a) 
   }
   if (head >= a.n_heads) return;
 
-  double* A = reinterpret_cast<double*>(smem + warp * kSolveBytes);   // [32][kLda] lag Gram, then L
-  double* rhs = A + 32 * kLda;
+  constexpr int kLda = Solve<NV>::kLda;
+  double* A = reinterpret_cast<double*>(smem + warp * Solve<NV>::kBytes);   // [NV-1][kLda] lag Gram, then L
+  double* rhs = A + Solve<NV>::kRows * kLda;
   double* invd = rhs + 32;
 
   const int n = a.wmax + 1;   // vectors used: the target and wmax lags
@@ -309,7 +318,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) predict_kernel(PredictArgs a) 
 template <int D, int NV>
 cudaError_t launch_t(const PredictArgs& a, cudaStream_t s) {
   const int grid = (a.n_heads + kWarps - 1) / kWarps;
-  const size_t smem = kWarps * kSolveBytes;
+  const size_t smem = kWarps * Solve<NV>::kBytes;
   auto kern = predict_kernel<D, NV>;
   if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
   return launch_prio(kern, dim3(grid), dim3(kWarps * 32), smem, s, a);
