@@ -81,6 +81,8 @@ typedef enum { ASP_COEF_SOFTMAX = 0, ASP_COEF_RAW = 1 } asp_coef_mode;
 #define ASP_DEV_BAD_PAGE   0x2   /* a page-table entry outside [0, n_pages) was skipped */
 #define ASP_DEV_WAIT_LIMIT 0x4   /* a bounded shared-memory barrier wait ran out */
 #define ASP_DEV_TAIL_LIMIT 0x8   /* a tail longer than max_tail was truncated */
+#define ASP_DEV_SELECT     0x10  /* a selection output position past C was skipped (a first-digit
+                                    histogram that does not match the scores) */
 
 /* The KV cache of one layer.
  *   page_size == 0: k, v are [batch, n_kv_heads, t_max, head_dim] (contiguous).

@@ -8,6 +8,7 @@ from ._lib import (  # noqa: F401
     ASP_F32,
     ASP_DEV_BAD_INDEX,
     ASP_DEV_BAD_PAGE,
+    ASP_DEV_SELECT,
     ASP_DEV_TAIL_LIMIT,
     ASP_DEV_WAIT_LIMIT,
     AspError,

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libasp.so")
 ASP_OK, ASP_ERR_INVALID_ARG, ASP_ERR_UNSUPPORTED, ASP_ERR_WORKSPACE, ASP_ERR_CUDA, ASP_ERR_TIMEOUT, ASP_ERR_DEVICE = range(7)
 ASP_F32, ASP_BF16 = 0, 1
 ASP_COEF_SOFTMAX, ASP_COEF_RAW = 0, 1
-ASP_DEV_BAD_INDEX, ASP_DEV_BAD_PAGE, ASP_DEV_WAIT_LIMIT, ASP_DEV_TAIL_LIMIT = 1, 2, 4, 8
+ASP_DEV_BAD_INDEX, ASP_DEV_BAD_PAGE, ASP_DEV_WAIT_LIMIT, ASP_DEV_TAIL_LIMIT, ASP_DEV_SELECT = 1, 2, 4, 8, 16
 
 # every entry point of include/asp.h with its ctypes signature
 class AspKv(ctypes.Structure):

@@ -50,6 +50,8 @@ struct AttParams {
   const int32_t* tail_begin;
   int max_tail;
   int splits, rows_per_split;
+  int n_items;   // units * splits: the persistent kernel's work items
+  int ctas;      // its grid
   float* part_o;
   float* part_ml;
   void* out;
@@ -454,8 +456,17 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
   const int g = lane >> 2, t = lane & 3;          // fragment row (query head) and column pair
   uint8_t* wbuf = smem + (size_t)warp * STAGES * TILE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kWarps * STAGES * TILE_BYTES) + warp * STAGES;
+  if (lane == 0) {
+    for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
 
-  const int unit = blockIdx.y, split = blockIdx.x;
+  // A persistent grid: each CTA takes work items (unit, split) in turn; the stage
+  // barriers' phases run on over the items (tbase: this warp's tiles so far).
+  uint32_t tbase = 0;
+  for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+  const int unit = item / p.splits, split = item - unit * p.splits;
   const int b = unit / p.n_kv, h = unit - b * p.n_kv;
   int T = p.seq_lens ? p.seq_lens[b] : p.t_max;
   T = T < 0 ? 0 : (T > p.t_max ? p.t_max : T);
@@ -476,12 +487,6 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
   const int r1 = min(n_rows, r0 + p.rows_per_split);
   const int n_tiles = r1 > r0 ? (r1 - r0 + kTile - 1) / kTile : 0;
   const int32_t* idx_row = n_sel ? p.idx + (size_t)unit * p.C : nullptr;
-
-  if (lane == 0) {
-    for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
-    mbar_init_fence();
-  }
-  __syncwarp();
 
   // query fragments: head g (zero rows for g >= G), channels 16kk + 2t (+8)
   uint32_t qa[KS][2];
@@ -571,7 +576,8 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
   int issued = 0;
 #pragma unroll 1
   for (int s = 0; s < STAGES && s < my_tiles; ++s) {
-    vmask[s] = issue(resolve(s), s);
+    const int sl = (int)((tbase + s) % STAGES);
+    vmask[sl] = issue(resolve(s), sl);
     ++issued;
   }
   RowSrc next = issued < my_tiles ? resolve(issued) : RowSrc{nullptr, false};
@@ -580,8 +586,8 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
   bool ok = true;
 #pragma unroll 1
   for (int tt = 0; tt < my_tiles; ++tt) {
-    const int slot = tt % STAGES;
-    ok = __all_sync(0xffffffffu, mbar_wait(&bars[slot], (uint32_t)(tt / STAGES) & 1u));
+    const int slot = (int)((tbase + tt) % STAGES);
+    ok = __all_sync(0xffffffffu, mbar_wait(&bars[slot], (uint32_t)((tbase + tt) / STAGES) & 1u));
     if (!ok) break;
     ++consumed;
     const uint32_t vm = vmask[slot];
@@ -646,7 +652,8 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
     }
   }
   if (!ok) {
-    for (int k = consumed + 1; k < issued; ++k) mbar_wait(&bars[k % STAGES], (uint32_t)(k / STAGES) & 1u);
+    for (int k = consumed + 1; k < issued; ++k)
+      mbar_wait(&bars[(tbase + k) % STAGES], (uint32_t)((tbase + k) / STAGES) & 1u);
   }
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
@@ -693,6 +700,11 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
         p.part_ml[(bh * p.splits + split) * 2 + 1] = L;
       }
     }
+  }
+  // the next item's copies overwrite the merge area: generic accesses first
+  fence_proxy_async_smem();
+  tbase += (uint32_t)my_tiles;
+  if (__syncthreads_or(!ok)) break;   // a wait ran out: stop (the copies have drained)
   }
 }
 
@@ -748,7 +760,7 @@ cudaError_t launch_mma(const AttParams& p, cudaStream_t s) {
   const size_t merge = (size_t)kWarps * G * (D + 2) * 4;
   if (smem < merge) smem = merge;
   if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
-  kern<<<dim3(p.splits, p.batch * p.n_kv), kWarps * 32, smem, s>>>(p);
+  kern<<<dim3(p.ctas), kWarps * 32, smem, s>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || p.splits == 1) return e;
   return launch_pdl(attend_merge_kernel<__nv_bfloat16, D>, dim3(p.batch * p.n_q_heads), dim3(D), 0, s,
@@ -785,7 +797,7 @@ cudaError_t dispatch_g(int G, const AttParams& p, cudaStream_t s) {
 // pure function of the sizes, so the workspace size is known without a device.
 AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail,
                        int ctas_per_sm) {
-  AttendPlan pl{1, 64, 0};
+  AttendPlan pl{1, 64, 0, 1};
   const long rows = (long)C + (max_tail > 0 ? max_tail : 0);
   const long units = (long)batch * n_kv_heads;
   if (rows <= 0 || units <= 0 || n_kv_heads <= 0) return pl;
@@ -798,6 +810,7 @@ AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, i
   per = ((per + quantum - 1) / quantum) * quantum;
   pl.rows_per_split = (int)per;
   pl.splits = (int)((rows + per - 1) / per);
+  pl.ctas = (int)(units * pl.splits < target ? units * pl.splits : target);   // at most one wave
   if (pl.splits > 1) {
     const size_t o = (size_t)batch * n_q_heads * pl.splits * head_dim * 4;
     const size_t ml = (size_t)batch * n_q_heads * pl.splits * 2 * 4;
@@ -829,6 +842,8 @@ cudaError_t launch_attend(const void* q, int q_f32, int n_q_heads, const KvView&
   p.tail_begin = tail_begin;
   p.max_tail = tail_begin ? max_tail : 0;
   p.splits = plan.splits;
+  p.n_items = plan.splits * kv.batch * kv.n_kv;
+  p.ctas = plan.ctas > 0 ? plan.ctas : 1;
   p.rows_per_split = plan.rows_per_split;
   if (plan.splits > 1) {
     const size_t o = (size_t)kv.batch * n_q_heads * plan.splits * kv.head_dim * 4;

@@ -481,7 +481,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) score_tc_kernel(const __grid_co
 // its group's 2G columns.  The B operand changes only with the sequence, so it
 // lives in two buffers outside the stages: the producer rewrites a buffer at a
 // sequence change once the MMAs that read its previous contents are complete.
-constexpr int kPageStages = 4;
+constexpr int kPageStages = 3;   // with two B buffers: fits beside a step-attention CTA
 constexpr int kPageHkv = 8;
 
 __host__ __device__ constexpr uint32_t tmem_alloc_cols(int cols) {

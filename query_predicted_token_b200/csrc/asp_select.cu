@@ -453,7 +453,12 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     const int Ej = run_eq + __popc(be & lt_mask);
     if (gt || (eq && Ej < krem)) {
       const int u = packed ? (int)(e & ~kGtTag) : w0 + k;
-      write_unit(u, Gj + min(Ej, krem));
+      const int pos = Gj + min(Ej, krem);
+      if (pos < a.c_units) {
+        write_unit(u, pos);
+      } else {   // only reachable with a histogram that does not match the scores
+        flag_status(ASP_DEV_SELECT);
+      }
       if (u == n - 1) s_last_sel = 1;
     }
     run_gt += __popc(bg);
