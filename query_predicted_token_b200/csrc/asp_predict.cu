@@ -94,7 +94,7 @@ struct GramRows {
 };
 
 template <int D, int NV>
-__global__ void __launch_bounds__(kWarps * 32, 1) predict_kernel(PredictArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(PredictArgs a) {
   constexpr int CPL = D / 32;   // contiguous channels per lane
   extern __shared__ __align__(16) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
