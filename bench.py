@@ -466,9 +466,9 @@ def main():
             if e2e:
                 q_t.copy_(q_host, non_blocking=True)
             st.step(q_t, out, lse)
-            s_main.wait_event(st.ev_sel_done)
-            if e2e:
+            if e2e:   # the output is ready when the attention ends: read it back while the selection runs
                 out_host.copy_(out, non_blocking=True)
+            s_main.wait_event(st.ev_sel_done)
             if k is not None:
                 ev[k][1].record(s_main)
 
