@@ -40,10 +40,12 @@ struct Solve {
 
 // 1/sqrt(x) for x > 0 in fp64: the fp32 hardware estimate refined by one
 // Newton-Raphson step y <- y (3 - x y^2) / 2, which squares its relative error
-// (about 1e-7 -> 1e-14) at the cost of four fp64 operations.
+// (about 1e-7 -> 1e-14); written as y + y (1/2 - (x/2) y^2), x/2 formed beside the
+// estimate, so three dependent fp64 operations follow it.
 __device__ __forceinline__ double rsqrt_f64(double x) {
+  const double hx = 0.5 * x;
   const double y = (double)rsqrtf((float)x);
-  return y * (1.5 - 0.5 * x * y * y);
+  return fma(y, fma(-hx * y, y, 0.5), y);
 }
 
 // Stores the reduced pair `q` (lane's pair of a round) into the solve arrays:
@@ -157,57 +159,63 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
 
   const int wm = a.wmax;
   constexpr int WMAX = NV - 1;   // lags the registers can hold
-  // Cholesky A = L L^T with lane i holding row i of the lower triangle in
-  // registers; the pivot comes from lane k by a shuffle, column k through shared
-  // memory.
+  // Cholesky A = L L^T fused with the forward substitution L z = rhs.  Lane i
+  // holds row i of A (then of L) and rhs_i (then z_i) in registers.  The chain
+  // that bounds the loop is pivot -> 1/L_kk -> the next pivot: lane k+1 forms its
+  // updated diagonal from its own entry L_{k+1,k} and sends it round by one
+  // shuffle, ahead of the rest of the column update (whose entries L_jk go through
+  // shared memory, one store per lane and one broadcast load per later column).
+  double z = lane < wm ? rhs[lane] : 0.0;
+  double* col = invd + 32;
   {
     double arow[WMAX];
 #pragma unroll
     for (int j = 0; j < WMAX; ++j) arow[j] = (j <= lane && lane < wm && j < wm) ? A[lane * kLda + j] : 0.0;
+    double piv = __shfl_sync(0xffffffffu, arow[0], 0);
+    double my_inv = 1.0;   // 1 / L_ii of this lane's row
 #pragma unroll
     for (int k = 0; k < WMAX; ++k) {
       if (k < wm) {
-        const double akk = __shfl_sync(0xffffffffu, arow[k], k);
-        const double inv = rsqrt_f64(akk);   // 1 / L_kk
-        const double dkk = akk * inv;        // L_kk = sqrt(A_kk)
+        const double inv = rsqrt_f64(piv);   // 1 / L_kk
         const double lik = (lane > k && lane < wm) ? arow[k] * inv : 0.0;
+        if (k + 1 < WMAX) {
+          const double dn = fma(-lik, lik, arow[k + 1]);   // lane k+1: A_{k+1,k+1} - L_{k+1,k}^2
+          piv = __shfl_sync(0xffffffffu, dn, k + 1);
+        }
+        const double zk = __shfl_sync(0xffffffffu, z, k) * inv;   // z_k
         if (lane == k) {
-          arow[k] = dkk;
+          my_inv = inv;
           invd[k] = inv;
+          z = zk;
         } else if (lane > k) {
           arow[k] = lik;
+          z = fma(-lik, zk, z);
         }
-        // column k goes through shared memory: one store per lane and one broadcast
-        // load per later column, instead of two shuffles per later column
-        double* col = invd + 32;
         col[lane] = lik;
         __syncwarp();
 #pragma unroll
         for (int j = k + 1; j < WMAX; ++j) {
           const double ljk = col[j];
-          if (j < wm && lane >= j && lane < wm) arow[j] -= lik * ljk;
+          if (j < wm && lane >= j && lane < wm) arow[j] = fma(-lik, ljk, arow[j]);
         }
         __syncwarp();   // the next column overwrites col
       }
     }
+    // rows of L scaled by their own 1 / L_ii: the back substitutions then need one
+    // multiply-add per step
     if (lane < wm) {
 #pragma unroll
       for (int j = 0; j < WMAX; ++j)
-        if (j <= lane) A[lane * kLda + j] = arow[j];
+        if (j < lane) A[lane * kLda + j] = arow[j] * my_inv;
     }
   }
   __syncwarp();
-  // forward substitution L z = rhs (shared by every window): lane i keeps z_i
-  double z = lane < wm ? rhs[lane] : 0.0;
-  for (int k = 0; k < wm; ++k) {
-    const double zk = __shfl_sync(0xffffffffu, z, k) * invd[k];
-    if (lane == k) z = zk;
-    if (lane > k && lane < wm) z -= A[lane * kLda + k] * zk;
-  }
   // Back substitutions L_w^T a = z_w for all windows at once: window wi owns the
-  // lanes [base_wi, base_wi + w) (in rounds if the widths exceed 32).  The
-  // weights are folded into beta_r = sum_w alpha_{w,r}, so that
-  // qhat = (1/|windows|) sum_r beta_r q_{t-r}.
+  // lanes [base_wi, base_wi + w) (in rounds if the widths exceed 32).  With
+  // y_k = z_k - sum_{j>k} L_jk a_j (complete once step k is reached) and
+  // a_k = y_k / L_kk, lane i < k takes y_k from lane k and subtracts
+  // (L_ki / L_kk) y_k.  The weights are folded into beta_r = sum_w alpha_{w,r},
+  // so that qhat = (1/|windows|) sum_r beta_r q_{t-r}.
   double* beta = rhs;   // rhs is no longer needed: reuse it for beta
   if (lane < 32) beta[lane] = 0.0;
   __syncwarp();
@@ -230,12 +238,26 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
     double av = (my_w > 0) ? __shfl_sync(0xffffffffu, z, li) : __shfl_sync(0xffffffffu, z, 0);
     int kmax = 0;
     for (int k = first; k < last; ++k) kmax = max(kmax, win[k]);
-    for (int k = kmax - 1; k >= 0; --k) {
-      const bool act = k < my_w;
-      const double ak = __shfl_sync(0xffffffffu, av, act ? my_base + k : lane) * invd[k];
-      if (act && li == k) av = ak;
-      if (act && li < k) av -= A[k * kLda + li] * ak;
+    if constexpr (WMAX <= 16) {
+      // the lane's column of the scaled factor in registers, then a chain of
+      // one shuffle and one multiply-add per step
+      double lt[WMAX];
+#pragma unroll
+      for (int k = 0; k < WMAX; ++k) lt[k] = (li < k && k < my_w) ? A[k * kLda + li] : 0.0;
+#pragma unroll
+      for (int k = WMAX - 1; k >= 0; --k) {
+        if (k < kmax) {
+          const double yk = __shfl_sync(0xffffffffu, av, k < my_w ? my_base + k : lane);
+          if (li < k && k < my_w) av = fma(-lt[k], yk, av);
+        }
+      }
+    } else {
+      for (int k = kmax - 1; k >= 0; --k) {
+        const double yk = __shfl_sync(0xffffffffu, av, k < my_w ? my_base + k : lane);
+        if (li < k && k < my_w) av = fma(-A[k * kLda + li], yk, av);
+      }
     }
+    if (my_w > 0) av *= invd[li];   // a_li
     if (a.win_fast) {
       // Windows of 2^j lanes at multiples of their width: maxima and sums over a
       // window are xor butterflies, and lag r gathers its weights by shuffles.
