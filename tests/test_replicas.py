@@ -13,6 +13,7 @@ import multiprocessing as mp
 import os
 import socket
 import sys
+import time
 
 import pytest
 
@@ -56,6 +57,15 @@ def _rank_main(rank: int, world: int, port: int, q) -> None:
         q.put((rank, "error", repr(e), None, None, None))
 
 
+def _send_and_exit(q, item, code: int) -> None:
+    """Puts ``item`` and ends the process at once; the queue's feeder thread is
+    joined first, or ``os._exit`` can end the process before the message is out."""
+    q.put(item)
+    q.close()
+    q.join_thread()
+    os._exit(code)
+
+
 def _rank_dies(rank: int, world: int, port: int, q) -> None:
     """Rank 1 exits abruptly after joining (no teardown, so its sockets close at
     once); rank 0 then enters a collective."""
@@ -64,19 +74,16 @@ def _rank_dies(rank: int, world: int, port: int, q) -> None:
         g = ReplicaGroup("gloo", "cpu", timeout_s=30)
         g.barrier()   # both ranks fully connected before one of them leaves
     except Exception as e:
-        q.put((rank, "setup failed", repr(e)))
-        os._exit(1)
+        _send_and_exit(q, (rank, "setup failed", repr(e)), 1)
     if rank == 1:
-        q.put((rank, "raised", None))
-        q.close()
-        q.join_thread()   # the message is out before the process ends
-        os._exit(3)
+        _send_and_exit(q, (rank, "raised", None), 3)
+    t0 = time.monotonic()   # start-up time (spawn, imports) is not what is tested: time the collective
     try:
         g.slowest(1.0)
-        q.put((rank, "no error", None))
+        item = (rank, "no error", time.monotonic() - t0)
     except Exception as e:
-        q.put((rank, "error", type(e).__name__))
-    os._exit(0)   # the group is broken: skip its teardown
+        item = (rank, "error", type(e).__name__, time.monotonic() - t0)
+    _send_and_exit(q, item, 0)   # the group is broken: skip its teardown
 
 
 def _run(target, world: int = 2, join_s: float = 120.0):
@@ -147,6 +154,7 @@ def test_two_gloo_ranks_aggregate():
 def test_dead_rank_ends_collective_with_error():
     # the survivor's collective fails when the dead rank's sockets close, well inside
     # the group's 30 s timeout
-    res = _run(_rank_dies, join_s=90.0)
+    res = _run(_rank_dies, join_s=120.0)
     assert res[1][1] == "raised"
     assert res[0][1] == "error", res[0]
+    assert res[0][3] < 60.0, res[0]   # within the 30 s process-group timeout, with margin
