@@ -95,7 +95,9 @@ struct GramRows {
   }
 };
 
-template <int D, int NV>
+// FAST: the windows are powers of two that fit one warp (PredictArgs::win_fast);
+// the kernel for that case carries no code for the general one.
+template <int D, int NV, bool FAST>
 __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(PredictArgs a) {
   constexpr int CPL = D / 32;   // contiguous channels per lane
   extern __shared__ __align__(16) uint8_t smem[];
@@ -258,7 +260,7 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
       }
     }
     if (my_w > 0) av *= invd[li];   // a_li
-    if (a.win_fast) {
+    if constexpr (FAST) {
       // Windows of 2^j lanes at multiples of their width: maxima and sums over a
       // window are xor butterflies, and lag r gathers its weights by shuffles.
       float w32 = my_w > 0 ? (float)av : 0.f;
@@ -323,7 +325,7 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
   float acc[CPL];
 #pragma unroll
   for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
-  const float bl = lane < WMAX ? (a.win_fast ? bfast : (float)beta[lane]) : 0.f;
+  const float bl = lane < WMAX ? (FAST ? bfast : (float)beta[lane]) : 0.f;
 #pragma unroll
   for (int r = 0; r < NV - 1; ++r) {   // lag r (q_{t-1-r}) weights q_{t-r} = h[r]
     const float br = __shfl_sync(0xffffffffu, bl, r);
@@ -341,7 +343,7 @@ template <int D, int NV>
 cudaError_t launch_t(const PredictArgs& a, cudaStream_t s) {
   const int grid = (a.n_heads + kWarps - 1) / kWarps;
   const size_t smem = kWarps * Solve<NV>::kBytes;
-  auto kern = predict_kernel<D, NV>;
+  auto kern = a.win_fast ? predict_kernel<D, NV, true> : predict_kernel<D, NV, false>;
   if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
   return launch_prio(kern, dim3(grid), dim3(kWarps * 32), smem, s, a);
 }

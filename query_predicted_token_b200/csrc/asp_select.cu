@@ -78,6 +78,9 @@ __device__ __forceinline__ int cta_exclusive_scan(int x, int* wsum, int* total) 
   return excl;
 }
 
+// FUSED: the first digit's histogram is given and the scores load as 16-byte
+// vectors (the decode step's case); that kernel carries no code for the others.
+template <bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.x;
@@ -132,7 +135,11 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   const bool vec = (a.row_stride & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0;
   // With the first histogram given, the threshold digit is found while the row's
   // scores load, and the units are classified and packed straight from registers.
-  const bool fused = !own_h0 && vec && a.key_cap >= kWarps * 4;
+  const bool fused = FUSED;
+  if (FUSED && !(!own_h0 && vec && a.key_cap >= kWarps * 4)) {   // the launch rule was not met
+    if (tid == 0) flag_status(ASP_DEV_SELECT);
+    return;
+  }
   const bool keys_in_smem = cached && !fused;   // the key array is built (else keys are re-read from L2)
   auto key_at = [&](int i) -> uint32_t { return keys_in_smem ? keys[i] : order_key(srow[i]); };
   if (!fused && cached && vec) {
@@ -478,8 +485,11 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   // shared-memory slots for keys or packed lists; the same for every row
   args.key_cap = len_max <= kSmemKeys ? ((len_max + 3) & ~3) : kSmemKeys;
   const size_t smem = (size_t)(args.key_cap > 0 ? args.key_cap : 4) * 4;
-  if (prepare_kernel((const void*)select_kernel, smem, kThreads) < 1) return cudaErrorInvalidConfiguration;
-  return launch_pdl(select_kernel, dim3(args.n_rows), dim3(kThreads), smem, s, args);
+  const bool fused = a.hist0 != nullptr && (a.row_stride & 3) == 0 &&
+                     (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0 && args.key_cap >= kWarps * 4;
+  auto kern = fused ? select_kernel<true> : select_kernel<false>;
+  if (prepare_kernel((const void*)kern, smem, kThreads) < 1) return cudaErrorInvalidConfiguration;
+  return launch_pdl(kern, dim3(args.n_rows), dim3(kThreads), smem, s, args);
 }
 
 ASP_STATUS_READER(read_status_select)
