@@ -204,6 +204,31 @@ def test_decode_selection_of_tied_scores_keeps_the_first_tokens():
             assert np.all(idx[b, h, n:] == -1)
 
 
+def test_decode_selection_ties_across_the_halves_of_a_row():
+    """Two-valued scores: a set of tokens, most of them in the second half of the
+    row, scores one value and every other token the other (0.0).  When the first
+    half alone cannot fill the quota, the lowest-index rule for tied tokens carries
+    into the second half.  With few rows each row is split over two CTAs, so the
+    second CTA's output positions depend on the first's counts; the result must
+    equal the oracle's selection over the same scores, index for index."""
+    B, Hkv, G, d, T, C = 2, 2, 2, 128, 16384, 12000
+    lens = torch.tensor([16384, 13001], dtype=torch.int32)
+    g = torch.Generator().manual_seed(11)
+    u = torch.randn(d, generator=g)
+    k = torch.zeros(B, Hkv, T, d)
+    marked = torch.zeros(T, dtype=torch.bool)
+    marked[9000::7] = True           # second half, strided
+    marked[15000:15500] = True       # a block near the end
+    marked[100:140] = True           # a few in the first half
+    k[:, :, marked] = u
+    k = k.to(torch.bfloat16).to(DEV)
+    v = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).to(DEV)
+    scores, idx, cnt = _decode_once(k, v, lens, Hkv * G, C)
+    ref_idx, ref_cnt = oracle.select_topk(scores, lens.tolist(), C)
+    assert np.array_equal(cnt, ref_cnt)
+    assert np.array_equal(idx, ref_idx)
+
+
 def test_decode_selection_when_most_tokens_survive_the_first_digit():
     """C close to T_b on rows longer than the selection's shared memory: the survivors
     of the first digit overflow the packed lists and the row is re-read from L2."""
