@@ -33,7 +33,6 @@ constexpr int kSmemKeys = 48 * 1024;   // 192 KB of keys
 constexpr int kBins = kTopBins;        // widest digit: 11 bits
 constexpr int kBpt = kBins / kThreads;
 constexpr uint32_t kGtTag = 0x80000000u;
-constexpr int kPairMinUnits = 8192;    // rows at least this long may take two CTAs
 
 // The float whose order key is k (see order_key), for a bin edge k: a NaN
 // pattern below the key of -inf gives -inf, one above the key of +inf gives NaN
@@ -79,41 +78,12 @@ __device__ __forceinline__ int cta_exclusive_scan(int x, int* wsum, int* total) 
   return excl;
 }
 
-// Pairs of CTAs (a cluster of two) on one row: rank, barrier, and loads from the
-// partner's shared memory.
-__device__ __forceinline__ int cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return (int)r;
-}
-// Every thread of both CTAs arrives; shared-memory writes before it (atomics
-// included) are visible to the partner after it.
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t partner_addr(const void* p, int rank) {
-  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ int ld_partner(uint32_t addr) {
-  int v;
-  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-
 // FUSED: the first digit's histogram is given and the scores load as 16-byte
 // vectors (the decode step's case); that kernel carries no code for the others.
-// P = 2 (FUSED only): a cluster of two CTAs per row, each on a contiguous half of
-// the units; the later digits' histograms are summed through the partner's shared
-// memory, and the second CTA's output positions start after the first's.
-template <bool FUSED, int P>
+template <bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  static_assert(P == 1 || (P == 2 && FUSED), "pairs run the fused path only");
-  const int row = P == 2 ? (int)blockIdx.x >> 1 : (int)blockIdx.x;
-  const int rank = P == 2 ? cluster_rank() : 0;
+  const int row = blockIdx.x;
   const int b = row / a.rows_per_seq;
   pdl_wait();   // the scores (and their histogram) come from the previous kernel
 
@@ -122,7 +92,6 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   __shared__ int wsum[kWarps];
   __shared__ int wg[kWarps], we[kWarps];
   __shared__ int s_digit, s_above, s_bincnt, s_last_sel, s_overflow;
-  __shared__ int s_tot_gt, s_tot_eq;   // this CTA's units above / at the threshold
 
   int T = a.seq_lens ? a.seq_lens[b] : a.t_max;
   T = T < 0 ? 0 : (T > a.t_max ? a.t_max : T);
@@ -138,21 +107,14 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     }
   };
 
-  if (n <= a.c_units) {   // every unit chosen (by the first CTA of a pair)
-    if (rank == 0) {
-      for (int u = tid; u < n; u += kThreads) write_unit(u, u);
-      for (int i = n * E + tid; i < out_stride; i += kThreads) out[i] = -1;
-      if (tid == 0) a.count[row] = T;
-    }
+  if (n <= a.c_units) {   // every unit chosen
+    for (int u = tid; u < n; u += kThreads) write_unit(u, u);
+    for (int i = n * E + tid; i < out_stride; i += kThreads) out[i] = -1;
+    if (tid == 0) a.count[row] = T;
     return;
   }
-  // this CTA's units [lo_r, hi_r): the whole row, or a half (a multiple of 4 units,
-  // so that 16-byte loads stay aligned)
-  const int H = P == 2 ? (((n + 1) / 2 + 3) & ~3) : n;
-  const int lo_r = min(n, rank * H), hi_r = min(n, lo_r + H);
-  const int n_loc = hi_r > lo_r ? hi_r - lo_r : 0;
 
-  const bool cached = n_loc <= a.key_cap;   // this CTA's units fit the shared-memory slots
+  const bool cached = n <= a.key_cap;   // the whole row fits the shared-memory slots
   const float* srow = a.scores + (size_t)row * a.row_stride;
 
   // ---- load the keys (cached rows) and, without a given first histogram, count the top digit
@@ -255,15 +217,15 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   };
 
   // Warp w owns the contiguous units [w0, w1) (in 128-unit chunks when fused).
-  const int R = fused ? ((((n_loc + kWarps - 1) / kWarps) + 127) & ~127) : ((((n + kWarps - 1) / kWarps) + 31) & ~31);
-  const int w0 = min(hi_r, lo_r + warp * R), w1 = min(hi_r, w0 + R);
+  const int R = fused ? ((((n + kWarps - 1) / kWarps) + 127) & ~127) : ((((n + kWarps - 1) / kWarps) + 31) & ~31);
+  const int w0 = min(n, warp * R), w1 = min(n, w0 + R);
   const uint32_t lt_mask = (1u << lane) - 1u;
   // Warp w's packed list lives in the slots [pb, pe): its own range when the row
   // fits, else an equal share of the slots (a longer list overflows it, and the
   // row falls back to re-reading its scores in every pass).
   const int share = (a.key_cap / kWarps) & ~3;
-  const int pb = (fused && !cached) ? warp * share : w0 - lo_r;
-  const int pe = (fused && !cached) ? pb + share : w1 - lo_r;
+  const int pb = (fused && !cached) ? warp * share : w0;
+  const int pe = (fused && !cached) ? pb + share : w1;
   int* h1 = hist[1];
   int n_packed = 0;
   bool done;
@@ -359,10 +321,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
       __syncthreads();
     }
     if (!done && !packed) {   // overflow: count the candidates from the scores
-      for (int base = lo_r; base < hi_r; base += kThreads) {
+      for (int base = 0; base < n; base += kThreads) {
         const int i = base + tid;
-        const uint32_t key = i < hi_r ? order_key(srow[i]) : 0u;
-        count_digit(h1, i < hi_r && (key & mask0) == prefix0, (key >> 10) & 2047u);
+        const uint32_t key = i < n ? order_key(srow[i]) : 0u;
+        count_digit(h1, i < n && (key & mask0) == prefix0, (key >> 10) & 2047u);
       }
       __syncthreads();
     }
@@ -411,16 +373,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   };
 
   // ---- second (11 bits) and third (10 bits) digits
-  if (!done) {   // the same in both CTAs of a pair: they found the same first digit
-    int* h1s = h1;
-    if constexpr (P == 2) {   // the pair's sum, in hist[0] (the partner reads h1 meanwhile)
-      cluster_sync();
-      const uint32_t ph = partner_addr(h1, rank ^ 1);
-      for (int i = tid; i < kBins; i += kThreads) hist[0][i] = h1[i] + ld_partner(ph + 4u * (uint32_t)i);
-      __syncthreads();
-      h1s = hist[0];
-    }
-    done = find_digit(h1s, 2048, 10);
+  if (!done) {
+    done = find_digit(h1, 2048, 10);
     if (!done) {
       int* h2 = hist[0];
       for (int i = tid; i < 1024; i += kThreads) h2[i] = 0;
@@ -433,22 +387,14 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
           count_digit(h2, !(e & kGtTag) && (key & mask) == prefix, key & 1023u);
         }
       } else {
-        for (int base = lo_r; base < hi_r; base += kThreads) {
+        for (int base = 0; base < n; base += kThreads) {
           const int i = base + tid;
-          const uint32_t key = i < hi_r ? key_at(i) : 0u;
-          count_digit(h2, i < hi_r && (key & mask) == prefix, key & 1023u);
+          const uint32_t key = i < n ? key_at(i) : 0u;
+          count_digit(h2, i < n && (key & mask) == prefix, key & 1023u);
         }
       }
       __syncthreads();
-      int* h2s = h2;
-      if constexpr (P == 2) {   // the partner has read h1 by now: the pair's sum goes there
-        cluster_sync();
-        const uint32_t ph = partner_addr(h2, rank ^ 1);
-        for (int i = tid; i < 1024; i += kThreads) h1[i] = h2[i] + ld_partner(ph + 4u * (uint32_t)i);
-        __syncthreads();
-        h2s = h1;
-      }
-      find_digit(h2s, 1024, 0);
+      find_digit(h2, 1024, 0);
     }
   }
 
@@ -498,22 +444,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     }
     wg[lane] = gi - g;   // exclusive offsets of the warps
     we[lane] = ei - e;
-    if (lane == 31) {
-      s_tot_gt = gi;
-      s_tot_eq = ei;
-    }
     if (lane == 0) s_last_sel = 0;
   }
   __syncthreads();
-  int base_gt = 0, base_eq = 0;   // units of the row before this CTA's that are above / at the threshold
-  if constexpr (P == 2) {
-    cluster_sync();
-    if (rank == 1) {
-      base_gt = ld_partner(partner_addr(&s_tot_gt, 0));
-      base_eq = ld_partner(partner_addr(&s_tot_eq, 0));
-    }
-  }
-  int run_gt = wg[warp] + base_gt, run_eq = we[warp] + base_eq;
+  int run_gt = wg[warp], run_eq = we[warp];
   for (int k0 = 0; k0 < span; k0 += 32) {
     const int k = k0 + lane;
     const bool valid = k < span;
@@ -538,8 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     run_eq += __popc(be);
   }
   __syncthreads();
-  if (tid == 0 && lo_r <= n - 1 && n - 1 < hi_r) a.count[row] = out_stride - (s_last_sel ? (n * E - T) : 0);
-  if constexpr (P == 2) cluster_sync();   // the partner's loads from this CTA are complete
+  if (tid == 0) a.count[row] = out_stride - (s_last_sel ? (n * E - T) : 0);
 }
 
 }  // namespace
@@ -554,21 +487,7 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)(args.key_cap > 0 ? args.key_cap : 4) * 4;
   const bool fused = a.hist0 != nullptr && (a.row_stride & 3) == 0 &&
                      (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0 && args.key_cap >= kWarps * 4;
-  // Two CTAs per row when the pairs still fit one wave and the rows are long
-  // enough for the halves to pay for the pair's exchanges.
-  if (fused && 2 * (long)a.n_rows <= sm_count() && len_max >= kPairMinUnits) {
-    SelectArgs pa = args;
-    const int half = ((len_max + 1) / 2 + 3) & ~3;
-    pa.key_cap = half <= kSmemKeys ? half : kSmemKeys;
-    const size_t psmem = (size_t)pa.key_cap * 4;
-    auto kern = select_kernel<true, 2>;
-    if (prepare_kernel((const void*)kern, psmem, kThreads) >= 1) {
-      const cudaError_t e = launch_pdl_cluster(kern, dim3(2 * a.n_rows), dim3(kThreads), psmem, s, 2u, pa);
-      if (e == cudaSuccess) return e;
-      (void)cudaGetLastError();   // a cluster that cannot be placed: one CTA per row below
-    }
-  }
-  auto kern = fused ? select_kernel<true, 1> : select_kernel<false, 1>;
+  auto kern = fused ? select_kernel<true> : select_kernel<false>;
   if (prepare_kernel((const void*)kern, smem, kThreads) < 1) return cudaErrorInvalidConfiguration;
   return launch_pdl(kern, dim3(args.n_rows), dim3(kThreads), smem, s, args);
 }

@@ -206,11 +206,10 @@ def test_decode_selection_of_tied_scores_keeps_the_first_tokens():
 
 def test_decode_selection_ties_across_the_halves_of_a_row():
     """Two-valued scores: a set of tokens, most of them in the second half of the
-    row, scores one value and every other token the other (0.0).  When the first
-    half alone cannot fill the quota, the lowest-index rule for tied tokens carries
-    into the second half.  With few rows each row is split over two CTAs, so the
-    second CTA's output positions depend on the first's counts; the result must
-    equal the oracle's selection over the same scores, index for index."""
+    row, scores one value and every other token the other (0.0).  The quota of tied
+    tokens (lowest index first) runs past the middle of the row, across the warps'
+    ranges and the warp-offset scan; the result must equal the oracle's selection
+    over the same scores, index for index."""
     B, Hkv, G, d, T, C = 2, 2, 2, 128, 16384, 12000
     lens = torch.tensor([16384, 13001], dtype=torch.int32)
     g = torch.Generator().manual_seed(11)
