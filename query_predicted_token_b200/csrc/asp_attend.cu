@@ -810,7 +810,12 @@ AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, i
   per = ((per + quantum - 1) / quantum) * quantum;
   pl.rows_per_split = (int)per;
   pl.splits = (int)((rows + per - 1) / per);
-  pl.ctas = (int)(units * pl.splits < target ? units * pl.splits : target);   // at most one wave
+  // The decode step's plan (ctas_per_sm given) runs its items, all of about C rows,
+  // as a persistent grid of at most one wave.  Otherwise one CTA per item: the
+  // rows of a tail can be as ragged as the sequences, and the hardware's CTA
+  // scheduling balances those better than a fixed stride over the items.
+  const long items = units * pl.splits;
+  pl.ctas = (int)(ctas_per_sm > 0 && items > target ? target : items);
   if (pl.splits > 1) {
     const size_t o = (size_t)batch * n_q_heads * pl.splits * head_dim * 4;
     const size_t ml = (size_t)batch * n_q_heads * pl.splits * 2 * 4;
