@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--layers", type=int, default=1,
                     help="also time a stack of this many layers (each with its own cache), steady-state period")
+    ap.add_argument("--side-streams", type=int, default=1,
+                    help="with --layers: side streams the layers' selection chains alternate over")
     return ap.parse_args()
 
 
@@ -349,13 +351,15 @@ def recall_analysis(wl, kv, dev):
 
 
 # ----------------------------------------------------------------------------- multi-layer stack
-def multi_layer_period(wl, layers, tokens, dev):
+def multi_layer_period(wl, layers, tokens, dev, side_streams=1):
     """Steady-state decode period of a stack of `layers` layers, each with its own
     cache and query history: per token, layer l's attention runs on the main stream
-    in layer order, and every layer's prediction, scan and selection run on one
-    shared side stream (the cache side of the pages' two ranks).  The period is the
-    time of `tokens` tokens over `tokens`, after 2 warm-up tokens; a layer is only
-    allocated while the device keeps 20% more memory free than it needs."""
+    in layer order, and layer l's prediction, scan and selection run on side stream
+    l mod `side_streams` (the cache side of the pages' two ranks; with two streams,
+    one layer's latency-bound prediction and selection can overlap the next
+    layer's scan).  The period is the time of `tokens` tokens over `tokens`, after
+    2 warm-up tokens; a layer is only allocated while the device keeps 20% more
+    memory free than it needs."""
     import torch
     import query_predicted_token_b200 as asp
     import synth
@@ -363,7 +367,7 @@ def multi_layer_period(wl, layers, tokens, dev):
     e = 2 if wl.kv_dtype == "bf16" else 4
     per_layer = 2 * B * Hkv * wl.t_max * d * e
     main_s = torch.cuda.current_stream()
-    side_s = torch.cuda.Stream(priority=-100)
+    side = [torch.cuda.Stream(priority=-100) for _ in range(max(1, side_streams))]
     states, outs, qs = [], [], []
     for l in range(layers):
         free, _ = torch.cuda.mem_get_info(dev)
@@ -374,7 +378,7 @@ def multi_layer_period(wl, layers, tokens, dev):
         kv = asp.KV(kvd["k"], kvd["v"], kvd["seq_lens"], kvd["page_table"], t_max=wl.t_max)
         qhist, q_next = synth.query_history(wl_l, steps=1)
         st = asp.DecodeState(kv, Hq, asp.PredCfg(wl.W, wl.windows, wl.lam), C, qhist.to(dev).contiguous(),
-                             s_main=main_s, s_side=side_s)
+                             s_main=main_s, s_side=side[l % len(side)])
         lens = kvd["seq_lens"].cpu().tolist()
         idx0, cnt0 = synth.random_selection(B, Hkv, C, lens, seed=wl_l.seed + 99)
         st.set_selection(idx0.to(dev), cnt0.to(dev))
@@ -397,16 +401,19 @@ def multi_layer_period(wl, layers, tokens, dev):
     a.record(main_s)
     for _ in range(tokens):
         token()
-    main_s.wait_event(states[-1].ev_sel_done)   # the last layer's selection ends the window
+    for st in states[-len(side):]:   # the last selection of every side stream ends the window
+        main_s.wait_event(st.ev_sel_done)
     b.record(main_s)
     torch.cuda.synchronize()
     period_us = a.elapsed_time(b) * 1e3 / tokens
     lens = synth.workloads.sequence_lengths(wl).tolist()
     step_b = step_bytes(wl, lens)["total"]
-    res = {"layers": n, "requested_layers": layers, "tokens": tokens, "period_us": round(period_us, 1),
+    res = {"layers": n, "requested_layers": layers, "side_streams": len(side), "tokens": tokens,
+           "period_us": round(period_us, 1),
            "per_layer_us": round(period_us / n, 2), "gbs": round(step_b * n / (period_us / 1e6) / 1e9, 1),
            "note": "per token: attention of every layer on the main stream in layer order, prediction, scan and "
-                   "selection of every layer on one side stream; no model weights or other layers' compute"}
+                   "selection of layer l on side stream l mod side_streams; no model weights or other layers' "
+                   "compute"}
     del states
     torch.cuda.empty_cache()
     return res
@@ -508,7 +515,8 @@ def main():
     # the pages' two baselines on the same cache and query: page-level selection, full attention
     compare = None if args.no_compare else comparison_paths(wl, kvd, kv, q_t, s_main, flush, args.steps)
     recall = None if args.no_compare else recall_analysis(wl, kv, dev)
-    stack = multi_layer_period(wl, args.layers, args.steps, dev) if args.layers > 1 else None
+    stack = (multi_layer_period(wl, args.layers, args.steps, dev, args.side_streams)
+             if args.layers > 1 else None)
     if stack and compare and stack.get("layers"):
         for k in ("page_level", "full_attention"):   # one layer's measured step times the layer count
             stack[k + "_period_us_from_one_layer"] = round(compare[k]["step_us"] * stack["layers"], 1)
