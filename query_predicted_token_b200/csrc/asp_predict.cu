@@ -96,8 +96,9 @@ struct GramRows {
 };
 
 // FAST: the windows are powers of two that fit one warp (PredictArgs::win_fast);
-// the kernel for that case carries no code for the general one.
-template <int D, int NV, bool FAST>
+// the kernel for that case carries no code for the general one.  EXACT: the
+// widest window has NV - 1 lags, so every bound on the lags is a constant.
+template <int D, int NV, bool FAST, bool EXACT>
 __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(PredictArgs a) {
   constexpr int CPL = D / 32;   // contiguous channels per lane
   extern __shared__ __align__(16) uint8_t smem[];
@@ -117,7 +118,8 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
   double* rhs = A + Solve<NV>::kRows * kLda;
   double* invd = rhs + 32;
 
-  const int n = a.wmax + 1;   // vectors used: the target and wmax lags
+  const int wmax = EXACT ? NV - 1 : a.wmax;   // lags of the widest window
+  const int n = wmax + 1;                      // vectors used: the target and wmax lags
   const int nslot = a.W + 1;
   float* hist = a.qhist + (size_t)head * nslot * D;
   const int start = a.q_new ? a.ring_start + 1 : a.ring_start;
@@ -128,7 +130,9 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
 #pragma unroll
     for (int c = 0; c < CPL; ++c) h[v][c] = 0.f;
     if (v < n) {
-      const int slot = (start + a.W - v) % nslot;
+      // start <= nslot and 0 <= W - v <= W < nslot: one subtraction wraps the slot
+      int slot = start + a.W - v;
+      if (slot >= nslot) slot -= nslot;
       float* src = hist + (size_t)slot * D + lane * CPL;
       if (v == 0 && a.q_new) {
         const size_t off = (size_t)head * D + lane * CPL;
@@ -155,12 +159,12 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
   // per round; after the reduce-scatter lane l holds pair (round base + l).
   {
     float part[32];
-    GramRows<NV, CPL, 0>::run(h, part, lane, a.wmax, a.lam, A, rhs);
+    GramRows<NV, CPL, 0>::run(h, part, lane, wmax, a.lam, A, rhs);
   }
   __syncwarp();
 
-  const int wm = a.wmax;
   constexpr int WMAX = NV - 1;   // lags the registers can hold
+  const int wm = wmax;
   // Cholesky A = L L^T fused with the forward substitution L z = rhs.  Lane i
   // holds row i of A (then of L) and rhs_i (then z_i) in registers.  The chain
   // that bounds the loop is pivot -> 1/L_kk -> the next pivot: lane k+1 forms its
@@ -343,7 +347,9 @@ template <int D, int NV>
 cudaError_t launch_t(const PredictArgs& a, cudaStream_t s) {
   const int grid = (a.n_heads + kWarps - 1) / kWarps;
   const size_t smem = kWarps * Solve<NV>::kBytes;
-  auto kern = a.win_fast ? predict_kernel<D, NV, true> : predict_kernel<D, NV, false>;
+  const bool exact = a.wmax == NV - 1;
+  auto kern = a.win_fast ? (exact ? predict_kernel<D, NV, true, true> : predict_kernel<D, NV, true, false>)
+                         : (exact ? predict_kernel<D, NV, false, true> : predict_kernel<D, NV, false, false>);
   if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
   return launch_prio(kern, dim3(grid), dim3(kWarps * 32), smem, s, a);
 }
