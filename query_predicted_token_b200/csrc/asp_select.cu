@@ -180,18 +180,17 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   // keys, given this CTA's histogram h (or the row's global one).
   uint32_t prefix = 0u, mask = 0u;
   int krem = a.c_units;
-  auto find_digit = [&](const int* h, int nb, int shift) -> bool {
+  // This thread's bins of a histogram, highest digit first.
+  auto bins_of = [&](const int* h, int nb, int (&v)[kBpt]) {
     const int bpt = nb / kThreads;
-    int v[kBpt];
+#pragma unroll
+    for (int j = 0; j < kBpt; ++j) v[j] = j < bpt ? h[nb - 1 - (tid * bpt + j)] : 0;
+  };
+  auto find_digit_in = [&](const int (&v)[kBpt], int nb, int shift) -> bool {
+    const int bpt = nb / kThreads;
     int local = 0;
 #pragma unroll
-    for (int j = 0; j < kBpt; ++j) {
-      v[j] = 0;
-      if (j < bpt) {
-        v[j] = h[nb - 1 - (tid * bpt + j)];
-        local += v[j];
-      }
-    }
+    for (int j = 0; j < kBpt; ++j) local += v[j];
     int total;
     const int excl = cta_exclusive_scan(local, wsum, &total);
     if (excl < krem && krem <= excl + local) {
@@ -214,6 +213,11 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     const bool done = s_bincnt == krem;
     __syncthreads();
     return done;
+  };
+  auto find_digit = [&](const int* h, int nb, int shift) -> bool {
+    int v[kBpt];
+    bins_of(h, nb, v);
+    return find_digit_in(v, nb, shift);
   };
 
   // Warp w owns the contiguous units [w0, w1) (in 128-unit chunks when fused).
@@ -248,10 +252,18 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
         f[u] = i < w1 ? ld_issue(s4 + (i >> 2)) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     };
+    // the histogram's bins are requested ahead of the scores, so that they do not
+    // queue behind the row's loads
+    static_assert(kBpt == 2, "two bins of the first digit per thread");
+    int hv[kBpt];
+    {   // bins 2047 - 2 tid and 2046 - 2 tid: one 8-byte load, kept ahead of the row's loads
+      const int* hp = a.hist0 + (size_t)row * kBins + (kBins - 2 - 2 * tid);
+      asm volatile("ld.global.v2.s32 {%0, %1}, [%2];" : "=r"(hv[1]), "=r"(hv[0]) : "l"(hp));
+    }
     load_chunks(w0);
     for (int i = tid; i < kBins; i += kThreads) h1[i] = 0;   // ordered by find_digit's barriers
     if (tid == 0) s_overflow = 0;
-    done = find_digit(a.hist0 + (size_t)row * kBins, 2048, kTopShift);
+    done = find_digit_in(hv, 2048, kTopShift);
     prefix0 = prefix;
     mask0 = mask;
     // The bin's edges as floats: a unit survives (is above the bin or in it) iff
