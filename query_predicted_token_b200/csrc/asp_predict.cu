@@ -223,27 +223,48 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
   // (L_ki / L_kk) y_k.  The weights are folded into beta_r = sum_w alpha_{w,r},
   // so that qhat = (1/|windows|) sum_r beta_r q_{t-r}.
   double* beta = rhs;   // rhs is no longer needed: reuse it for beta
-  if (lane < 32) beta[lane] = 0.0;
-  __syncwarp();
+  if constexpr (!FAST) {
+    beta[lane] = 0.0;
+    __syncwarp();
+  }
   int win[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) win[k] = a.windows[k];
   float bfast = 0.f;   // beta of lag `lane` on the fast path
   for (int first = 0; first < a.n_win;) {
-    int last = first, used = 0;   // windows [first, last) share this round
-    while (last < a.n_win && used + win[last] <= 32) used += win[last++];
-    int my_w = 0, my_base = 0, base = 0;
-    for (int k = first; k < last; ++k) {
-      if (lane >= base && lane < base + win[k]) {
-        my_w = win[k];
-        my_base = base;
+    int last = first;   // windows [first, last) share this round
+    int my_w = 0, my_base = 0, kmax = 0;
+    if constexpr (FAST) {
+      // one round holds every window; loops over a constant bound keep win[] in
+      // registers
+      last = a.n_win;
+      int base = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (k < last) {
+          if (lane >= base && lane < base + win[k]) {
+            my_w = win[k];
+            my_base = base;
+          }
+          base += win[k];
+          kmax = max(kmax, win[k]);
+        }
       }
-      base += win[k];
+    } else {
+      int used = 0;
+      while (last < a.n_win && used + win[last] <= 32) used += win[last++];
+      int base = 0;
+      for (int k = first; k < last; ++k) {
+        if (lane >= base && lane < base + win[k]) {
+          my_w = win[k];
+          my_base = base;
+        }
+        base += win[k];
+        kmax = max(kmax, win[k]);
+      }
     }
     const int li = lane - my_base;   // this lane's lag index in its window
     double av = (my_w > 0) ? __shfl_sync(0xffffffffu, z, li) : __shfl_sync(0xffffffffu, z, 0);
-    int kmax = 0;
-    for (int k = first; k < last; ++k) kmax = max(kmax, win[k]);
     if constexpr (WMAX <= 16) {
       // the lane's column of the scaled factor in registers, then a chain of
       // one shuffle and one multiply-add per step
@@ -285,10 +306,13 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
         w32 = my_w > 0 ? ex / zs : 0.f;
       }
       int bb = 0;
-      for (int k = first; k < last; ++k) {
-        const float v = __shfl_sync(0xffffffffu, w32, bb + (lane < win[k] ? lane : 0));
-        if (lane < win[k]) bfast += v;
-        bb += win[k];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (k < last) {
+          const float v = __shfl_sync(0xffffffffu, w32, bb + (lane < win[k] ? lane : 0));
+          if (lane < win[k]) bfast += v;
+          bb += win[k];
+        }
       }
       first = last;
       continue;
