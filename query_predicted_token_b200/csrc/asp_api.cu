@@ -337,6 +337,13 @@ asp_status asp_decode_step(const asp_decode_args* a) {
     e = asp::launch_append(kv, a->k_new, a->v_new, const_cast<int32_t*>(a->kv->seq_lens),
                            const_cast<int32_t*>(a->tail_begin), a->quest_meta, a->quest_page, sm);
   if (e == cudaSuccess) e = cudaEventRecord(fork, sm);
+  // main stream: attention of this step, issued first so that its CTAs (one per
+  // SM) are placed before the side chain's, in a captured graph as in a stream
+  if (e == cudaSuccess) e = mark(6, sm);
+  if (e == cudaSuccess)
+    e = asp::launch_attend(a->q_t, a->q_dtype == ASP_F32, a->n_q_heads, kv, a->idx_cur, a->count_cur, a->C,
+                           a->tail_begin, a->max_tail, a->out, a->lse, a->workspace, plan, sm);
+  if (e == cudaSuccess) e = mark(7, sm);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(ss, fork, 0);
   // side stream: selection for the next step
   if (e == cudaSuccess) e = mark(0, ss);
@@ -371,12 +378,6 @@ asp_status asp_decode_step(const asp_decode_args* a) {
   }
   if (e == cudaSuccess) e = mark(5, ss);
   if (e == cudaSuccess) e = cudaEventRecord(done, ss);
-  // main stream: attention of this step
-  if (e == cudaSuccess) e = mark(6, sm);
-  if (e == cudaSuccess)
-    e = asp::launch_attend(a->q_t, a->q_dtype == ASP_F32, a->n_q_heads, kv, a->idx_cur, a->count_cur, a->C,
-                           a->tail_begin, a->max_tail, a->out, a->lse, a->workspace, plan, sm);
-  if (e == cudaSuccess) e = mark(7, sm);
   return cuda_status(e);
 }
 
