@@ -512,6 +512,24 @@ def main():
         one_step(k, e2e=True)
     torch.cuda.synchronize()
     e2e_ms = [a.elapsed_time(b) for a, b in ev]
+    # The key scan alone, for its roofline: the same kernel and grid through
+    # asp_score_keys, launched back to back between two CUDA events on its stream
+    # (the keys are larger than L2 and read with an evict-first hint, so each launch
+    # streams them from HBM; one event pair per launch would add its ~6 µs floor).
+    # The per-kernel events inside the step also hold the launch gap after the
+    # predictor (events stop the programmatic dependent launch): `in_step_frac`.
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s_main):
+        flush.zero_()
+        for _ in range(2):
+            asp.score_keys(st.qpred, kv, st.scores, stream=s_main)
+        a0.record(s_main)
+        for _ in range(args.steps):
+            asp.score_keys(st.qpred, kv, st.scores, stream=s_main)
+        a1.record(s_main)
+    torch.cuda.synchronize()
+    assert asp.device_status() == 0
+    scan_alone_ms = a0.elapsed_time(a1) / args.steps
     # the pages' two baselines on the same cache and query: page-level selection, full attention
     compare = None if args.no_compare else comparison_paths(wl, kvd, kv, q_t, s_main, flush, args.steps)
     recall = None if args.no_compare else recall_analysis(wl, kv, dev)
@@ -528,7 +546,8 @@ def main():
     e2e_value = total_bytes / t_e2e / 1e9
     peak, peak_kind = read_peaks()
     score_ms = statistics.mean(kern_ms["score"])
-    achieved = acct["score"] / (score_ms / 1e3) / 1e9
+    in_step = acct["score"] / (score_ms / 1e3) / 1e9
+    achieved = acct["score"] / (scan_alone_ms / 1e3) / 1e9
     traffic = read_traffic("asp_score_tc.cu", 1.0) if wl.name == "qwen3_8b_shaped_32k" else None
 
     if rank == 0:
@@ -553,7 +572,12 @@ def main():
             "step_bytes": acct["total"],
             "roofline": {"kernel": "score_tc_kernel (key scan)", "bound": "hbm", "achieved": round(achieved, 1),
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "traffic": traffic, "algorithmic_bytes": acct["score"]},
+                         "traffic": traffic, "algorithmic_bytes": acct["score"],
+                         "timed": f"alone: {args.steps} back-to-back launches of the same kernel and grid "
+                                  "through asp_score_keys between two CUDA events on its stream; keys larger "
+                                  "than L2, read with an evict-first hint",
+                         "us": round(scan_alone_ms * 1e3, 2),
+                         "in_step_frac": round(in_step / peak, 4)},
             "step_frac_of_peak": round(value / world / peak, 4),
             "clocks": clk,
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),
