@@ -51,33 +51,6 @@ __device__ __forceinline__ float4 ld_issue(const float4* p) {
   return v;
 }
 
-// Exclusive scan of one int per thread over the CTA; also returns the total.
-__device__ __forceinline__ int cta_exclusive_scan(int x, int* wsum, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = x;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) wsum[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int w = wsum[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    wsum[lane] = w;
-  }
-  __syncthreads();
-  const int excl = incl - x + (warp > 0 ? wsum[warp - 1] : 0);
-  *total = wsum[kWarps - 1];
-  __syncthreads();
-  return excl;
-}
-
 // FUSED: the first digit's histogram is given and the scores load as 16-byte
 // vectors (the decode step's case); that kernel carries no code for the others.
 template <bool FUSED>
@@ -191,8 +164,24 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
     int local = 0;
 #pragma unroll
     for (int j = 0; j < kBpt; ++j) local += v[j];
-    int total;
-    const int excl = cta_exclusive_scan(local, wsum, &total);
+    // exclusive prefix of `local` over the CTA with one barrier: warp totals go to
+    // wsum, then every warp scans the 32 totals itself
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int wincl = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wincl, o);
+      if (lane >= o) wincl += y;
+    }
+    const int wbase = __shfl_sync(0xffffffffu, wincl - wsum[lane], warp);   // sum over the earlier warps
+    const int excl = wbase + incl - local;
     if (excl < krem && krem <= excl + local) {
       int run = excl;
       for (int j = 0; j < bpt; ++j) {
@@ -206,13 +195,13 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
       }
     }
     __syncthreads();
+    // s_digit, s_above, s_bincnt and wsum are written again only after the next
+    // search's first barrier, which every thread reaches after these reads
     const int digit = s_digit;
     krem -= s_above;
     prefix |= (uint32_t)digit << shift;
     mask |= ((uint32_t)nb - 1u) << shift;
-    const bool done = s_bincnt == krem;
-    __syncthreads();
-    return done;
+    return s_bincnt == krem;
   };
   auto find_digit = [&](const int* h, int nb, int shift) -> bool {
     int v[kBpt];
