@@ -530,6 +530,23 @@ def main():
     torch.cuda.synchronize()
     assert asp.device_status() == 0
     scan_alone_ms = a0.elapsed_time(a1) / args.steps
+    # The sparse attention alone (its stand-alone plan, three CTAs per SM), the same
+    # way, over the step's current selection: the second roofline row.
+    sel_idx, sel_cnt = st.selection
+    att_ws = torch.empty(max(16, int(asp.lib().asp_attend_workspace_bytes(B, Hq, Hkv, d, C, 0))),
+                         dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(s_main):
+        flush.zero_()
+        for _ in range(2):
+            asp.sparse_attend(q_t, kv, sel_idx, sel_cnt, C, out, workspace=att_ws, stream=s_main)
+        a0.record(s_main)
+        for _ in range(args.steps):
+            asp.sparse_attend(q_t, kv, sel_idx, sel_cnt, C, out, workspace=att_ws, stream=s_main)
+        a1.record(s_main)
+    torch.cuda.synchronize()
+    assert asp.device_status() == 0
+    att_alone_ms = a0.elapsed_time(a1) / args.steps
+    att_bytes = int(sel_cnt.sum().item()) * 2 * d * (2 if wl.kv_dtype == "bf16" else 4)
     # the pages' two baselines on the same cache and query: page-level selection, full attention
     compare = None if args.no_compare else comparison_paths(wl, kvd, kv, q_t, s_main, flush, args.steps)
     recall = None if args.no_compare else recall_analysis(wl, kv, dev)
@@ -578,6 +595,13 @@ def main():
                                   "than L2, read with an evict-first hint",
                          "us": round(scan_alone_ms * 1e3, 2),
                          "in_step_frac": round(in_step / peak, 4)},
+            "roofline_attend": {"kernel": "attend_mma_kernel (sparse attention, stand-alone plan)", "bound": "hbm",
+                                "achieved": round(att_bytes / (att_alone_ms / 1e3) / 1e9, 1), "peak": peak,
+                                "peak_kind": peak_kind, "unit": "GB/s",
+                                "frac": round(att_bytes / (att_alone_ms / 1e3) / 1e9 / peak, 4),
+                                "algorithmic_bytes": att_bytes, "us": round(att_alone_ms * 1e3, 2),
+                                "timed": f"alone: {args.steps} back-to-back asp_sparse_attend launches over the "
+                                         "step's selection between two CUDA events"},
             "step_frac_of_peak": round(value / world / peak, 4),
             "clocks": clk,
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),
