@@ -3,12 +3,13 @@
 // out[b, hq] = sum_{j in S} softmax_j(q . k_j / sqrt(d)) v_j over S = selected u tail.
 //
 // HBM-bound gather (each selected K and V row read once, 256 B for bf16 d=128).
-//  * grid = (splits, batch * n_kv): a CTA takes a contiguous slice of one KV head's
-//    attended rows and computes all G query heads of the group, so a row is read
-//    once for the whole group;
-//  * a warp gathers 16 rows per tile: each of its 32 lanes issues one 1-D bulk
-//    copy (TMA) of a K row (lanes 0-15) or a V row (lanes 16-31) into the warp's
-//    stage, all counted on one mbarrier; STAGES tiles are in flight per warp;
+//  * work items (split, batch * n_kv): a CTA takes a contiguous slice of one KV
+//    head's attended rows and computes all G query heads of the group, so a row
+//    is read once for the whole group;
+//  * a warp gathers 16 rows per tile (K and V) into its stage, counted on one
+//    mbarrier, with STAGES tiles in flight per warp: the CUDA-core kernel (fp32)
+//    by one 1-D bulk copy (TMA) per lane, the tensor-core kernel (bf16) by
+//    16-byte cp.async copies, several rows per warp instruction;
 //  * logits: 16-byte shared-memory vectors per lane, packed FMAs, warp
 //    reduce-scatter over the row's lanes; online softmax in base 2 (log2 e folded
 //    into the query scale); V accumulated in fp32 registers;
@@ -51,6 +52,7 @@ struct AttParams {
   int max_tail;
   int splits, rows_per_split;
   int n_items;   // units * splits: the persistent kernel's work items
+  int lean;      // launch the kernel form with fewer registers
   int ctas;      // its grid
   float* part_o;
   float* part_ml;
@@ -441,7 +443,11 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, u
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-template <int D, int G, int STAGES>
+// LEAN: the row copies are issued from a partly unrolled loop, which keeps the
+// registers at the level that lets one CTA share an SM with the key scan's and the
+// predictor's (the decode step); the fully unrolled form keeps more copies in
+// flight where three CTAs share an SM (stand-alone calls).
+template <int D, int G, int STAGES, bool LEAN>
 __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
   constexpr int ROW_BYTES = D * 2;
   constexpr int STRIDE = ROW_BYTES + 16;          // padded row pitch in shared memory
@@ -457,7 +463,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
   uint8_t* wbuf = smem + (size_t)warp * STAGES * TILE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kWarps * STAGES * TILE_BYTES) + warp * STAGES;
   if (lane == 0) {
-    for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 32);   // one arrival per lane's copies
     mbar_init_fence();
   }
   __syncwarp();
@@ -543,20 +549,34 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
     }
     return RowSrc{src, valid};
   };
+  // The tile's 32 rows go in as 16-byte copies, several rows per warp instruction
+  // (chunk lane%CPR of row RPI*i + lane/CPR): a row-sized bulk copy per lane kept
+  // too few bytes in flight per SM.  Rows that are not valid are zero-filled
+  // (source size 0, nothing is read).  Each lane's copies arrive once on the
+  // stage's barrier (count 32).
   auto issue = [&](const RowSrc& rs, int slot) -> uint32_t {
-    const int rr = lane & 15;
-    const bool isv = lane >= 16;
+    constexpr int CPR = ROW_BYTES / 16;   // 16-byte chunks per row: 16 (d 128) or 8 (d 64)
+    constexpr int RPI = 32 / CPR;          // rows per warp instruction
     const uint32_t vm = __ballot_sync(0xffffffffu, rs.valid) & 0xffffu;
-    uint8_t* dst = wbuf + slot * TILE_BYTES + (isv ? HALF : 0) + rr * STRIDE;
-    if (!rs.valid) {
+    uint8_t* const tile = wbuf + slot * TILE_BYTES;
+    const uint32_t c16 = (uint32_t)(lane % CPR) * 16u;
+    auto copy_rows = [&](int i) {   // warp instruction i: rows RPI*i .. RPI*i + RPI - 1
+      const int ri = RPI * i + lane / CPR;   // 0-15 K rows, 16-31 V rows (row ri is resolved by lane ri)
+      const uint64_t src = __shfl_sync(0xffffffffu, reinterpret_cast<uint64_t>(rs.src), ri);
+      const int valid = __shfl_sync(0xffffffffu, rs.valid ? 1 : 0, ri);
+      const uint32_t dst = smem_u32(tile + (ri < 16 ? 0 : HALF) + (ri & 15) * STRIDE) + c16;
+      const uint64_t from = valid ? src + c16 : reinterpret_cast<uint64_t>(p.k);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(from), "r"(valid ? 16 : 0)
+                   : "memory");
+    };
+    if constexpr (LEAN) {
+#pragma unroll 2
+      for (int i = 0; i < 32 / RPI; ++i) copy_rows(i);
+    } else {
 #pragma unroll
-      for (int c = 0; c < ROW_BYTES / 16; ++c) reinterpret_cast<uint4*>(dst)[c] = make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < 32 / RPI; ++i) copy_rows(i);
     }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)__popc(vm) * 2u * ROW_BYTES);
-    __syncwarp();
-    if (rs.valid) bulk_g2s(dst, rs.src, ROW_BYTES, &bars[slot]);
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&bars[slot])) : "memory");
     return vm;
   };
 
@@ -755,7 +775,7 @@ template <int D, int G>
 cudaError_t launch_mma(const AttParams& p, cudaStream_t s) {
   constexpr int STAGES = 2;
   constexpr int TILE_BYTES = 2 * kTile * (D * 2 + 16);
-  auto kern = attend_mma_kernel<D, G, STAGES>;
+  auto kern = p.lean ? attend_mma_kernel<D, G, STAGES, true> : attend_mma_kernel<D, G, STAGES, false>;
   size_t smem = (size_t)kWarps * STAGES * TILE_BYTES + kWarps * STAGES * 8;
   const size_t merge = (size_t)kWarps * G * (D + 2) * 4;
   if (smem < merge) smem = merge;
@@ -797,7 +817,7 @@ cudaError_t dispatch_g(int G, const AttParams& p, cudaStream_t s) {
 // pure function of the sizes, so the workspace size is known without a device.
 AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail,
                        int ctas_per_sm) {
-  AttendPlan pl{1, 64, 0, 1};
+  AttendPlan pl{1, 64, 0, 1, ctas_per_sm > 0 ? 1 : 0};
   const long rows = (long)C + (max_tail > 0 ? max_tail : 0);
   const long units = (long)batch * n_kv_heads;
   if (rows <= 0 || units <= 0 || n_kv_heads <= 0) return pl;
@@ -849,6 +869,7 @@ cudaError_t launch_attend(const void* q, int q_f32, int n_q_heads, const KvView&
   p.splits = plan.splits;
   p.n_items = plan.splits * kv.batch * kv.n_kv;
   p.ctas = plan.ctas > 0 ? plan.ctas : 1;
+  p.lean = plan.lean;
   p.rows_per_split = plan.rows_per_split;
   if (plan.splits > 1) {
     const size_t o = (size_t)kv.batch * n_q_heads * plan.splits * kv.head_dim * 4;

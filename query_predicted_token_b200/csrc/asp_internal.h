@@ -151,6 +151,7 @@ struct AttendPlan {
   int rows_per_split;
   size_t workspace_bytes;
   int ctas;   // CTAs of the (persistent) tensor-core attention grid
+  int lean;   // 1: the kernel form with fewer registers (one CTA per SM beside the key scan)
 };
 // ctas_per_sm: resident CTAs per SM the grid is sized for (0: as many as fit).
 AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail,
