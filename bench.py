@@ -43,9 +43,12 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-compare", action="store_true",
                     help="skip the page-level and full-attention timings and the selection recall")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the records of the other decode workloads (32B shapes, ragged paged batch)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--layers", type=int, default=1,
-                    help="also time a stack of this many layers (each with its own cache), steady-state period")
+    ap.add_argument("--layers", type=int, default=36,
+                    help="also time a stack of this many layers (each with its own cache), steady-state period "
+                         "(1: no stack)")
     ap.add_argument("--side-streams", type=int, default=1,
                     help="with --layers: side streams the layers' selection chains alternate over")
     return ap.parse_args()
@@ -101,12 +104,12 @@ def read_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def read_traffic(kernel_file: str, launch_units: float):
-    """Per-launch DRAM bytes of the score kernel from the committed ncu summary, if it
-    was taken on the current source of that kernel (else None)."""
+def read_traffic(kernel_file: str, launch_units: float, summary: str = "score_keys_qwen3_8b_shaped_32k.txt"):
+    """Per-launch DRAM bytes of a kernel from its committed ncu summary (scaled by
+    ``launch_units``), if the summary was taken on the kernel's current source (else None)."""
     import hashlib
     src = os.path.join(ROOT, "query_predicted_token_b200", "csrc", kernel_file)
-    summ = os.path.join(ROOT, "profiles", "score_keys_qwen3_8b_shaped_32k.txt")
+    summ = os.path.join(ROOT, "profiles", summary)
     try:
         h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
         kv = {}
@@ -269,16 +272,230 @@ def run_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- timing helpers
+L2_BYTES = 126 << 20
+
+
+def rotation_count(bytes_per_launch: float) -> int:
+    """Copies of a kernel's input to rotate over, so that between two launches that
+    read the same copy the other launches stream at least twice the L2 through it:
+    no launch can find the rows of an earlier one in L2."""
+    return max(2, min(8, math.ceil(2 * L2_BYTES / max(1.0, bytes_per_launch)) + 1))
+
+
+def time_rotating(fn, copies, stream, reps):
+    """Mean µs per launch of ``fn(copy)`` over ``reps`` back-to-back launches that
+    cycle through ``copies``, between two CUDA events on ``stream``."""
+    import torch
+    with torch.cuda.stream(stream):
+        for c in copies:                       # every copy once, untimed
+            fn(c)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(reps):
+            fn(copies[i % len(copies)])
+        b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) * 1e3 / reps
+
+
+def time_cold(fn, stream, flush, reps):
+    """Median µs of single launches, each after an L2 flush (outside its events);
+    an event pair alone measures ~5-6 µs on this part, so this is an upper bound."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for k in range(reps):
+            flush.zero_()
+            ev[k][0].record(stream)
+            fn()
+            ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) * 1e3 for a, b in ev)
+
+
+def roofline_entry(kernel, nbytes, us_rot, us_cold, peak, peak_kind, timed, traffic=None, extra=None):
+    achieved = nbytes / (us_rot / 1e6) / 1e9
+    d = {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+         "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic, "algorithmic_bytes": int(nbytes),
+         "us": round(us_rot, 2), "cold_us": round(us_cold, 2),
+         "cold_frac": round(nbytes / (us_cold / 1e6) / 1e9 / peak, 4), "timed": timed}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def clone_kv(asp, kvd, wl, with_v=True):
+    """Another cache of the same shapes (values copied), for rotation."""
+    k2 = kvd["k"].clone()
+    v2 = kvd["v"].clone() if with_v else kvd["v"]
+    return asp.KV(k2, v2, kvd["seq_lens"], kvd["page_table"], t_max=wl.t_max), (k2, v2)
+
+
+# ----------------------------------------------------------------------------- one decode workload
+def decode_record(wl, dev, args, flush, peak, peak_kind, *, headline, group=None):
+    """Times the decode step of a workload and its two roofline kernels.
+
+    Returns (record, extras): the record for the JSON line; extras holds the objects
+    the headline reuses (cache, query, state) and the per-step e2e numbers."""
+    import torch
+    import query_predicted_token_b200 as asp
+    import synth
+    B, Hq, Hkv, d, C = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.C
+    e = 2 if wl.kv_dtype == "bf16" else 4
+    steps = args.steps if headline else max(3, min(args.steps, 10))
+    kvd = synth.kv_cache(wl, dev)
+    lens = kvd["seq_lens"].cpu().tolist()
+    paged = kvd["page_table"] is not None
+    tail = 1 if paged else 0
+    kv = asp.KV(kvd["k"], kvd["v"], kvd["seq_lens"], kvd["page_table"], t_max=wl.t_max)
+    qhist, q_next = synth.query_history(wl, steps=1)
+    q_host = q_next[0].to(wl.torch_dtype()).pin_memory()
+    q_t = q_host.to(dev)
+    tail_begin = (kvd["seq_lens"] - tail).clamp(min=0).to(torch.int32) if tail else None
+    snap = (torch.tensor(lens) - tail).tolist() if tail else lens
+    idx0, cnt0 = synth.random_selection(B, Hkv, C, snap, seed=wl.seed + 99)
+    st = asp.DecodeState(kv, Hq, asp.PredCfg(wl.W, wl.windows, wl.lam), C, qhist.to(dev).contiguous(),
+                         max_tail=tail, tail_begin=tail_begin, timing=True)
+    st.set_selection(idx0.to(dev), cnt0.to(dev))
+    out = torch.empty(B, Hq, d, dtype=wl.torch_dtype(), device=dev)
+    out_host = torch.empty_like(out, device="cpu").pin_memory()
+    lse = torch.empty(B, Hq, device=dev)
+    s_main = st.s_main
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    acct = step_bytes(wl, lens)
+
+    def one_step(state, k=None, e2e=False):
+        with torch.cuda.stream(s_main):
+            flush.zero_()                                   # L2 flush, outside the timed events
+            if k is not None:
+                ev[k][0].record(s_main)
+            if e2e:
+                q_t.copy_(q_host, non_blocking=True)
+            state.step(q_t, out, lse)
+            if e2e:   # the output is ready when the attention ends: read it back while the selection runs
+                out_host.copy_(out, non_blocking=True)
+            s_main.wait_event(state.ev_sel_done)
+            if k is not None:
+                ev[k][1].record(s_main)
+
+    for _ in range(max(3, args.warmup)):
+        one_step(st)
+    torch.cuda.synchronize()
+    if group is not None:
+        group.barrier()
+    # timed steps: no events between the kernels, so each kernel of the side
+    # stream may launch while the previous one drains
+    st.set_timing(False)
+    torch.cuda.synchronize()
+    for k in range(steps):
+        one_step(st, k)
+    torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    # the same steps again with events around every kernel, for the per-kernel times
+    kern_ms = {n: [] for n in ("predict", "score", "select", "attend")}
+    st.set_timing(True)
+    for k in range(steps):
+        one_step(st)
+        torch.cuda.synchronize()
+        te = st.timing_events
+        for i, n in enumerate(("predict", "score", "select", "attend")):
+            kern_ms[n].append(te[2 * i].elapsed_time(te[2 * i + 1]))
+    st.set_timing(False)
+    assert asp.device_status() == 0
+    e2e_ms = None
+    if headline:
+        for k in range(steps):
+            one_step(st, k, e2e=True)
+        torch.cuda.synchronize()
+        e2e_ms = [a.elapsed_time(b) for a, b in ev]
+    serial_us = None
+    if paged:
+        # the same kernels on one stream: what the side stream buys on one GPU
+        st1 = asp.DecodeState(kv, Hq, asp.PredCfg(wl.W, wl.windows, wl.lam), C, qhist.to(dev).contiguous(),
+                              max_tail=tail, tail_begin=tail_begin, s_main=s_main, s_side=s_main)
+        st1.set_selection(idx0.to(dev), cnt0.to(dev))
+        for _ in range(max(3, args.warmup)):
+            one_step(st1)
+        for k in range(steps):
+            one_step(st1, k)
+        torch.cuda.synchronize()
+        serial_us = statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e3
+        del st1
+    # ---- the key scan alone: the same kernel and grid through asp_score_keys,
+    # alternating between two copies of the keys
+    kv2, keep2 = clone_kv(asp, kvd, wl, with_v=False)
+
+    def scan(kvx):
+        asp.score_keys(st.qpred, kvx, st.scores, stream=s_main)
+    scan_rot = time_rotating(scan, [kv, kv2], s_main, max(10, steps))
+    scan_cold = time_cold(lambda: scan(kv), s_main, flush, max(10, steps))
+    del kv2, keep2
+    assert asp.device_status() == 0
+    # ---- the sparse attention alone (its stand-alone plan), rotating over copies of the cache
+    sel_idx, sel_cnt = st.selection
+    att_bytes = int(sel_cnt.sum().item()) * 2 * d * e + (B * Hkv * tail * 2 * d * e)
+    att_ws = torch.empty(max(16, int(asp.lib().asp_attend_workspace_bytes(B, Hq, Hkv, d, C, tail))),
+                         dtype=torch.uint8, device=dev)
+    R = rotation_count(att_bytes)
+    copies, keep = [kv], []
+    for _ in range(R - 1):
+        kvx, kk = clone_kv(asp, kvd, wl)
+        copies.append(kvx)
+        keep.append(kk)
+
+    def attend(kvx):
+        asp.sparse_attend(q_t, kvx, sel_idx, sel_cnt, C, out, None, tail_begin, tail, att_ws, stream=s_main)
+    att_rot = time_rotating(attend, copies, s_main, max(10, steps))
+    att_cold = time_cold(lambda: attend(kv), s_main, flush, max(10, steps))
+    del copies, keep
+    torch.cuda.empty_cache()
+    assert asp.device_status() == 0
+
+    step_us = statistics.mean(step_ms) * 1e3
+    gbs = acct["total"] / (step_us / 1e6) / 1e9
+    traffic = read_traffic("asp_score_tc.cu", 1.0) if wl.name == "qwen3_8b_shaped_32k" else None
+    rot_note = "back-to-back launches cycling through {n} copies of the {what} (no launch finds an earlier launch's data in L2)"
+    rec = {
+        "workload": wl.name,
+        "config": {"batch": B, "n_q_heads": Hq, "n_kv_heads": Hkv, "head_dim": d, "T": wl.t_max,
+                   "t_min": wl.t_min, "ragged": wl.ragged, "paged": paged, "C": C, "W": wl.W,
+                   "windows": list(wl.windows), "lambda": wl.lam, "tail": tail},
+        "steps": steps,
+        "step_us": round(step_us, 2),
+        "step_us_p90": round(sorted(step_ms)[int(0.9 * (len(step_ms) - 1))] * 1e3, 2),
+        "gbs": round(gbs, 1),
+        "step_bytes": acct["total"],
+        "step_frac_of_peak": round(gbs / peak, 4),
+        "ideal_step_us": round(acct["total"] / (peak * 1e9) * 1e6, 2),
+        "kernel_us": {n: round(statistics.mean(v) * 1e3, 2) for n, v in kern_ms.items()},
+        "roofline": roofline_entry("score_tc_kernel (key scan)", acct["score"], scan_rot, scan_cold, peak, peak_kind,
+                                   rot_note.format(n=2, what="keys") + "; cold: one launch after an L2 flush",
+                                   traffic=traffic,
+                                   extra={"in_step_frac": round(acct["score"] / (statistics.mean(kern_ms["score"]) / 1e3) / 1e9 / peak, 4)}),
+        "roofline_attend": roofline_entry("attend_gather_kernel (+ merge) (sparse attention, stand-alone plan)",
+                                          att_bytes, att_rot, att_cold, peak, peak_kind,
+                                          rot_note.format(n=R, what="K/V cache") + "; cold: one launch after an L2 flush"),
+    }
+    if serial_us is not None:
+        rec["serial_step_us"] = round(serial_us, 2)
+        rec["overlap_gain_us"] = round(serial_us - step_us, 2)
+    extras = dict(kvd=kvd, kv=kv, q_t=q_t, q_host=q_host, out=out, st=st, s_main=s_main, e2e_ms=e2e_ms,
+                  step_ms=step_ms, acct=acct, lens=lens,
+                  h2d=q_host.numel() * q_host.element_size(), d2h=out.numel() * out.element_size())
+    return rec, extras
+
+
 # ----------------------------------------------------------------------------- comparison paths
-def comparison_paths(wl, kvd, kv, q_dev, stream, flush, steps):
-    """Times, on the same cache and query, the page-level comparison path (page
-    bound scan and page choice with the current query, then attention over the
-    chosen pages' tokens) and full attention over every cached token.  The page
-    bounds are built once beforehand (a serving system keeps them up to date as
-    tokens arrive).  Returns a dict for the JSON line."""
+def page_level_record(wl, kvd, kv, q_dev, stream, flush, steps, peak, peak_kind):
+    """The page-level comparison path on the given cache and query: page bounds
+    scanned with the current query, the best ceil(C/16) pages kept, attention over
+    their tokens.  The bounds are built once beforehand (a serving system keeps them
+    current as tokens arrive).  Step time, and the page-bound scan's roofline."""
     import torch
     import query_predicted_token_b200 as asp
     B, Hq, Hkv, d, C = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.C
+    e = 2 if wl.kv_dtype == "bf16" else 4
     dev = kvd["k"].device
     lens = kvd["seq_lens"].cpu().tolist()
     npm = math.ceil(wl.t_max / QUEST_PAGE)
@@ -289,9 +506,6 @@ def comparison_paths(wl, kvd, kv, q_dev, stream, flush, steps):
     qcnt = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
     out = torch.empty(B, Hq, d, dtype=wl.torch_dtype(), device=dev)
     ws_q = torch.empty(max(16, asp.attend_workspace_bytes(B, Hq, Hkv, d, cp)), dtype=torch.uint8, device=dev)
-    zero = torch.zeros(B, dtype=torch.int32, device=dev)
-    ws_d = torch.empty(max(16, asp.attend_workspace_bytes(B, Hq, Hkv, d, 0, wl.t_max)), dtype=torch.uint8,
-                       device=dev)
     with torch.cuda.stream(stream):
         asp.quest_build_meta(kv, QUEST_PAGE, meta, stream=stream)
 
@@ -299,30 +513,62 @@ def comparison_paths(wl, kvd, kv, q_dev, stream, flush, steps):
         asp.quest_select(q_dev, kv, meta, QUEST_PAGE, C, ps, qidx, qcnt, stream=stream)
         asp.sparse_attend(q_dev, kv, qidx, qcnt, cp, out, workspace=ws_q, stream=stream)
 
-    def dense_step():
-        asp.sparse_attend(q_dev, kv, None, None, 0, out, None, zero, wl.t_max, ws_d, stream=stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for k in range(-3, steps):
+            flush.zero_()
+            if k >= 0:
+                ev[k][0].record(stream)
+            quest_step()
+            if k >= 0:
+                ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    nbytes = quest_step_bytes(wl, lens)
+    # the page-bound scan alone, rotating over copies of the bounds
+    scan_bytes = nbytes["scan"]
+    R = rotation_count(scan_bytes)
+    metas = [meta] + [meta.clone() for _ in range(R - 1)]
 
-    res = {}
-    for name, fn, nbytes in (("page_level", quest_step, quest_step_bytes(wl, lens)["total"]),
-                             ("full_attention", dense_step, dense_bytes(wl, lens))):
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-        with torch.cuda.stream(stream):
-            for k in range(-3, steps):
-                flush.zero_()
-                if k >= 0:
-                    ev[k][0].record(stream)
-                fn()
-                if k >= 0:
-                    ev[k][1].record(stream)
-        torch.cuda.synchronize()
-        ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-        res[name] = {"step_us": round(ms * 1e3, 2), "gbs": round(nbytes / (ms / 1e3) / 1e9, 1), "bytes": nbytes}
-    res["note"] = ("same cache, query and L2 flush; page_level: page bounds scanned with the current query, "
-                   f"{cp // QUEST_PAGE} pages of {QUEST_PAGE} kept, attention over their tokens; "
-                   "full_attention: every cached token")
-    return res
+    def bound_scan(m):
+        asp.quest_page_scores(q_dev, kv, m, QUEST_PAGE, ps, stream=stream)
+    scan_rot = time_rotating(bound_scan, metas, stream, max(10, steps))
+    scan_cold = time_cold(lambda: bound_scan(meta), stream, flush, max(10, steps))
+    del metas
+    assert asp.device_status() == 0
+    return {
+        "workload": "quest_page_scan_8b_32k",
+        "config": {"batch": B, "n_q_heads": Hq, "n_kv_heads": Hkv, "head_dim": d, "T": wl.t_max, "C": C,
+                   "page": QUEST_PAGE, "pages_kept": cp // QUEST_PAGE},
+        "step_us": round(ms * 1e3, 2), "gbs": round(nbytes["total"] / (ms / 1e3) / 1e9, 1),
+        "step_bytes": nbytes["total"], "step_frac_of_peak": round(nbytes["total"] / (ms / 1e3) / 1e9 / peak, 4),
+        "roofline": roofline_entry("score_tc_kernel<2d> (page-bound scan)", scan_bytes, scan_rot, scan_cold, peak,
+                                   peak_kind, f"back-to-back launches cycling through {R} copies of the page "
+                                   "bounds; cold: one launch after an L2 flush",
+                                   traffic=read_traffic("asp_score_tc.cu", 1.0, "score_page_bounds_qwen3_8b_shaped_32k.txt")),
+        "note": "same cache, query and L2 flush as the token-level step of this shape; the bounds are built once, "
+                "untimed; the attention over the chosen pages is the same kernel as the token-level path's",
+    }
 
 
+def full_attention_record(wl, kvd, kv, q_dev, stream, flush, steps, peak):
+    """Full attention over every cached token (the pages' other baseline), through
+    the tail path of asp_sparse_attend."""
+    import torch
+    import query_predicted_token_b200 as asp
+    B, Hq, Hkv, d = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+    dev = kvd["k"].device
+    lens = kvd["seq_lens"].cpu().tolist()
+    out = torch.empty(B, Hq, d, dtype=wl.torch_dtype(), device=dev)
+    zero = torch.zeros(B, dtype=torch.int32, device=dev)
+    ws_d = torch.empty(max(16, asp.attend_workspace_bytes(B, Hq, Hkv, d, 0, wl.t_max)), dtype=torch.uint8,
+                       device=dev)
+    us = time_cold(lambda: asp.sparse_attend(q_dev, kv, None, None, 0, out, None, zero, wl.t_max, ws_d,
+                                             stream=stream), stream, flush, steps)
+    nbytes = dense_bytes(wl, lens)
+    return {"step_us": round(us, 2), "gbs": round(nbytes / (us / 1e6) / 1e9, 1), "bytes": nbytes,
+            "frac_of_peak": round(nbytes / (us / 1e6) / 1e9 / peak, 4),
+            "note": "every cached token through the tail path of asp_sparse_attend; one launch after an L2 flush"}
 # ----------------------------------------------------------------------------- selection recall
 def recall_analysis(wl, kv, dev):
     """Recall of the true next query's top-C set (untimed): the step's own
@@ -420,6 +666,9 @@ def multi_layer_period(wl, layers, tokens, dev, side_streams=1):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+SUB_WORKLOADS = ("qwen3_32b_shaped_32k", "longcot_ragged_paged_b64")
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -439,177 +688,78 @@ def main():
     asp.lib()   # raises if the library is missing: there is no other path
     wl = rank_workload(synth.workload(args.workload), rank)   # each rank: its own batch
     B, Hq, Hkv, d, C = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.C
-    kvd = synth.kv_cache(wl, dev)
-    lens = kvd["seq_lens"].cpu().tolist()
-    paged = kvd["page_table"] is not None
-    tail = 1 if paged else 0
-    kv = asp.KV(kvd["k"], kvd["v"], kvd["seq_lens"], kvd["page_table"], t_max=wl.t_max)
-    qhist, q_next = synth.query_history(wl, steps=1)
-    q_host = q_next[0].to(wl.torch_dtype()).pin_memory()
-    q_t = q_host.to(dev)
-    tail_begin = (kvd["seq_lens"] - tail).clamp(min=0).to(torch.int32) if tail else None
-    snap = (torch.tensor(lens) - tail).tolist() if tail else lens
-    idx0, cnt0 = synth.random_selection(B, Hkv, C, snap, seed=wl.seed + 99)
-    st = asp.DecodeState(kv, Hq, asp.PredCfg(wl.W, wl.windows, wl.lam), C, qhist.to(dev).contiguous(),
-                         max_tail=tail, tail_begin=tail_begin, timing=True)
-    st.set_selection(idx0.to(dev), cnt0.to(dev))
-    out = torch.empty(B, Hq, d, dtype=wl.torch_dtype(), device=dev)
-    out_host = torch.empty_like(out, device="cpu").pin_memory()
-    lse = torch.empty(B, Hq, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    s_main = st.s_main
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    acct = step_bytes(wl, lens)
-    # the decode step's attention has a merge launch when its plan splits the rows:
-    # its workspace then holds partials before the histogram
-    dec_ws = int(asp.lib().asp_decode_workspace_bytes(B, Hq, Hkv, d, C, tail))
-    splits = dec_ws > B * Hkv * 2048 * 4
-
-    def one_step(k=None, e2e=False):
-        with torch.cuda.stream(s_main):
-            flush.zero_()                                   # L2 flush, outside the timed events
-            if k is not None:
-                ev[k][0].record(s_main)
-            if e2e:
-                q_t.copy_(q_host, non_blocking=True)
-            st.step(q_t, out, lse)
-            if e2e:   # the output is ready when the attention ends: read it back while the selection runs
-                out_host.copy_(out, non_blocking=True)
-            s_main.wait_event(st.ev_sel_done)
-            if k is not None:
-                ev[k][1].record(s_main)
-
-    for _ in range(max(3, args.warmup)):
-        one_step()
-    torch.cuda.synchronize()
-    group.barrier()
+    peak, peak_kind = read_peaks()
     gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
     gpu_id = gpu_id if gpu_id.startswith("GPU-") else "GPU-" + gpu_id
-    kern_ms = {n: [] for n in ("predict", "score", "select", "attend")}
     with ClockSampler(gpu_id) as clocks:
-        # timed steps: no events between the kernels, so each kernel of the side
-        # stream may launch while the previous one drains
-        st.set_timing(False)
-        torch.cuda.synchronize()
-        for k in range(args.steps):
-            one_step(k)
-        torch.cuda.synchronize()
-        step_ms = [a.elapsed_time(b) for a, b in ev]
-        # the same steps again with events around every kernel, for the per-kernel
-        # times and the scan's roofline
-        st.set_timing(True)
-        for k in range(args.steps):
-            one_step()
-            torch.cuda.synchronize()
-            te = st.timing_events
-            for i, n in enumerate(("predict", "score", "select", "attend")):
-                kern_ms[n].append(te[2 * i].elapsed_time(te[2 * i + 1]))
-        st.set_timing(False)
-        torch.cuda.synchronize()
-    assert asp.device_status() == 0
-    # e2e: host query in, host output back, every step
-    for k in range(args.steps):
-        one_step(k, e2e=True)
-    torch.cuda.synchronize()
-    e2e_ms = [a.elapsed_time(b) for a, b in ev]
-    # The key scan alone, for its roofline: the same kernel and grid through
-    # asp_score_keys, launched back to back between two CUDA events on its stream
-    # (the keys are larger than L2 and read with an evict-first hint, so each launch
-    # streams them from HBM; one event pair per launch would add its ~6 µs floor).
-    # The per-kernel events inside the step also hold the launch gap after the
-    # predictor (events stop the programmatic dependent launch): `in_step_frac`.
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(s_main):
-        flush.zero_()
-        for _ in range(2):
-            asp.score_keys(st.qpred, kv, st.scores, stream=s_main)
-        a0.record(s_main)
-        for _ in range(args.steps):
-            asp.score_keys(st.qpred, kv, st.scores, stream=s_main)
-        a1.record(s_main)
-    torch.cuda.synchronize()
-    assert asp.device_status() == 0
-    scan_alone_ms = a0.elapsed_time(a1) / args.steps
-    # The sparse attention alone (its stand-alone plan, three CTAs per SM), the same
-    # way, over the step's current selection: the second roofline row.
-    sel_idx, sel_cnt = st.selection
-    att_ws = torch.empty(max(16, int(asp.lib().asp_attend_workspace_bytes(B, Hq, Hkv, d, C, 0))),
-                         dtype=torch.uint8, device=dev)
-    with torch.cuda.stream(s_main):
-        flush.zero_()
-        for _ in range(2):
-            asp.sparse_attend(q_t, kv, sel_idx, sel_cnt, C, out, workspace=att_ws, stream=s_main)
-        a0.record(s_main)
-        for _ in range(args.steps):
-            asp.sparse_attend(q_t, kv, sel_idx, sel_cnt, C, out, workspace=att_ws, stream=s_main)
-        a1.record(s_main)
-    torch.cuda.synchronize()
-    assert asp.device_status() == 0
-    att_alone_ms = a0.elapsed_time(a1) / args.steps
-    att_bytes = int(sel_cnt.sum().item()) * 2 * d * (2 if wl.kv_dtype == "bf16" else 4)
-    # the pages' two baselines on the same cache and query: page-level selection, full attention
-    compare = None if args.no_compare else comparison_paths(wl, kvd, kv, q_t, s_main, flush, args.steps)
-    recall = None if args.no_compare else recall_analysis(wl, kv, dev)
-    stack = (multi_layer_period(wl, args.layers, args.steps, dev, args.side_streams)
-             if args.layers > 1 else None)
-    if stack and compare and stack.get("layers"):
-        for k in ("page_level", "full_attention"):   # one layer's measured step times the layer count
-            stack[k + "_period_us_from_one_layer"] = round(compare[k]["step_us"] * stack["layers"], 1)
-
-    t_rank, t_e2e = group.slowest(sum(step_ms) / 1e3, sum(e2e_ms) / 1e3)
-    (total_bytes,) = group.total(acct["total"] * args.steps)   # ragged batches differ per rank
+        head, x = decode_record(wl, dev, args, flush, peak, peak_kind, headline=True, group=group)
+        t_rank, t_e2e = group.slowest(sum(x["step_ms"]) / 1e3, sum(x["e2e_ms"]) / 1e3)
+        ms_per_step = statistics.mean(x["step_ms"])
+        io = (x["h2d"], x["d2h"])
+        (total_bytes,) = group.total(x["acct"]["total"] * args.steps)   # ragged batches differ per rank
+        group.barrier()
+        extra = {}
+        if world == 1 and not args.no_compare:
+            # the pages' two baselines on the same cache and query
+            extra["page_level"] = page_level_record(wl, x["kvd"], x["kv"], x["q_t"], x["s_main"], flush,
+                                                    max(5, min(args.steps, 20)), peak, peak_kind)
+            extra["full_attention"] = full_attention_record(wl, x["kvd"], x["kv"], x["q_t"], x["s_main"], flush,
+                                                            max(5, min(args.steps, 20)), peak)
+            extra["recall"] = recall_analysis(wl, x["kv"], dev)
+        del x
+        torch.cuda.empty_cache()
+        subs = {}
+        if world == 1 and not args.no_workloads:
+            for name in SUB_WORKLOADS:
+                rec, y = decode_record(synth.workload(name), dev, args, flush, peak, peak_kind, headline=False)
+                del y
+                torch.cuda.empty_cache()
+                subs[name] = rec
+        stack = None
+        if world == 1 and args.layers > 1:
+            stack = multi_layer_period(wl, args.layers, max(3, min(args.steps, 10)), dev, args.side_streams)
     group.barrier()
     value = total_bytes / t_rank / 1e9
     e2e_value = total_bytes / t_e2e / 1e9
-    peak, peak_kind = read_peaks()
-    score_ms = statistics.mean(kern_ms["score"])
-    in_step = acct["score"] / (score_ms / 1e3) / 1e9
-    achieved = acct["score"] / (scan_alone_ms / 1e3) / 1e9
-    traffic = read_traffic("asp_score_tc.cu", 1.0) if wl.name == "qwen3_8b_shaped_32k" else None
 
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             gbs, sample, n, t = time_oracle(wl, args.cpu_seconds)
             cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle", "sample": sample}
-        clk = clocks.summary()
+        if "page_level" in extra:
+            subs["quest_page_scan_8b_32k"] = extra["page_level"]
+        if stack and "page_level" in extra and stack.get("layers"):
+            # one layer's measured step times the layer count
+            stack["page_level_period_us_from_one_layer"] = round(extra["page_level"]["step_us"] * stack["layers"], 1)
+            stack["full_attention_period_us_from_one_layer"] = round(
+                extra["full_attention"]["step_us"] * stack["layers"], 1)
+        # the decode step's attention launches a merge when its plan splits the rows
+        dec_ws = int(asp.lib().asp_decode_workspace_bytes(B, Hq, Hkv, d, C, 0))
+        splits = dec_ws > B * Hkv * 2048 * 4
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": max(3, args.warmup), "ms_per_step": round(statistics.mean(step_ms), 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.kv_dtype == "bf16" else "f32",
-            "data": "synthetic",
-            "config": {"workload": wl.name, "batch": B, "n_q_heads": Hq, "n_kv_heads": Hkv, "head_dim": d,
-                       "T": wl.t_max, "ragged": wl.ragged, "paged": paged, "C": C, "W": wl.W,
-                       "windows": list(wl.windows), "lambda": wl.lam,
-                       "l2": "flushed before every step (512 MiB write outside the timed events); KV larger than L2",
-                       "parallelism": f"replicas x{world} (one decode batch per GPU, no collective)"},
-            "step_us": round(statistics.mean(step_ms) * 1e3, 2),
-            "step_us_p90": round(sorted(step_ms)[int(0.9 * (len(step_ms) - 1))] * 1e3, 2),
-            "kernel_us": {n: round(statistics.mean(v) * 1e3, 2) for n, v in kern_ms.items()},
-            "step_bytes": acct["total"],
-            "roofline": {"kernel": "score_tc_kernel (key scan)", "bound": "hbm", "achieved": round(achieved, 1),
-                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "traffic": traffic, "algorithmic_bytes": acct["score"],
-                         "timed": f"alone: {args.steps} back-to-back launches of the same kernel and grid "
-                                  "through asp_score_keys between two CUDA events on its stream; keys larger "
-                                  "than L2, read with an evict-first hint",
-                         "us": round(scan_alone_ms * 1e3, 2),
-                         "in_step_frac": round(in_step / peak, 4)},
-            "roofline_attend": {"kernel": "attend_mma_kernel (sparse attention, stand-alone plan)", "bound": "hbm",
-                                "achieved": round(att_bytes / (att_alone_ms / 1e3) / 1e9, 1), "peak": peak,
-                                "peak_kind": peak_kind, "unit": "GB/s",
-                                "frac": round(att_bytes / (att_alone_ms / 1e3) / 1e9 / peak, 4),
-                                "algorithmic_bytes": att_bytes, "us": round(att_alone_ms * 1e3, 2),
-                                "timed": f"alone: {args.steps} back-to-back asp_sparse_attend launches over the "
-                                         "step's selection between two CUDA events"},
+            "warmup": max(3, args.warmup), "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if wl.kv_dtype == "bf16" else "f32", "data": "synthetic",
+            "config": dict(head["config"], workload=wl.name,
+                           l2="flushed before every step (512 MiB write outside the timed events); KV larger than L2",
+                           parallelism=f"replicas x{world} (one decode batch per GPU, no collective)"),
+            "step_us": head["step_us"], "step_us_p90": head["step_us_p90"], "kernel_us": head["kernel_us"],
+            "step_bytes": head["step_bytes"], "ideal_step_us": head["ideal_step_us"],
+            "roofline": head["roofline"], "roofline_attend": head["roofline_attend"],
             "step_frac_of_peak": round(value / world / peak, 4),
-            "clocks": clk,
-            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),
-                    "d2h_bytes_per_step": out.numel() * out.element_size()},
+            "clocks": clocks.summary(),
+            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": io[0],
+                    "d2h_bytes_per_step": io[1]},
             "gpu_launches": args.steps * (4 + (1 if splits else 0)),
             "cpu_baseline": cpu,
-            "comparison": compare,
-            "selection_recall": recall,
+            "workloads": subs or None,
+            "comparison": {"full_attention": extra.get("full_attention"),
+                           "page_level_step_us": extra["page_level"]["step_us"] if "page_level" in extra else None}
+            if extra else None,
+            "selection_recall": extra.get("recall"),
             "multi_layer": stack,
         }
         print(json.dumps(line), flush=True)

@@ -126,7 +126,8 @@ typedef struct {
  * window).  For each query head and each window w: ridge-fit q_t on the lags
  * q_{t-w}..q_{t-1} over the head_dim channels, a = (X X^T + lambda I)^-1 X q_t,
  * turn a into weights (softmax or raw), apply weight i to q_{t-w+i}; average
- * the window predictions.  Gram, Cholesky solve and weights run in fp64.
+ * the window predictions.  The Gram matrix and right-hand side are formed in fp32;
+ * the Cholesky factorisation, both substitutions and the weights run in fp64.
  *
  * qhist : device fp32 ring [batch, n_q_heads, W+1, head_dim].  Slot
  *         (ring_start + s) % (W+1) holds the s-th oldest vector (s = 0..W).
@@ -192,8 +193,9 @@ ASP_API asp_status asp_select_topk(const float* scores, const int32_t* seq_lens,
  *              tail_begin = 0 and count = 0 gives dense attention.
  * out        : device [batch, n_q_heads, head_dim] in kv_dtype, written.
  * lse        : device fp32 [batch, n_q_heads] or NULL.
- * workspace  : device scratch of at least asp_attend_workspace_bytes(...) bytes
- *              (any alignment of 256 bytes); contents need no initialisation.
+ * workspace  : device scratch of at least asp_attend_workspace_bytes(...) bytes,
+ *              16-byte aligned; contents need no initialisation.  May be NULL when
+ *              asp_attend_workspace_bytes(...) is 0.
  * Errors: ASP_ERR_INVALID_ARG; ASP_ERR_UNSUPPORTED; ASP_ERR_WORKSPACE. */
 ASP_API asp_status asp_sparse_attend(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv,
                              const int32_t* idx, const int32_t* count, int C,
@@ -338,6 +340,14 @@ ASP_API asp_status asp_wait_selection(asp_event_t ev_sel_done, long timeout_us);
  *        per page and channel the minimum (index 0) and maximum (index 1) key value
  *        over the page's valid tokens. */
 ASP_API asp_status asp_quest_build_meta(const asp_kv* kv, int quest_page, void* meta, asp_stream_t stream);
+
+/* The page scores alone (the first half of asp_quest_select): page_scores
+ * [batch, n_kv_heads, ceil(t_max / quest_page)] fp32 get u_p (defined below) for
+ * every page holding a valid token; entries past a sequence's pages are not
+ * written.  Same arguments and errors as asp_quest_select, less the selection's. */
+ASP_API asp_status asp_quest_page_scores(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv,
+                                         const void* meta, int quest_page, float* page_scores,
+                                         asp_stream_t stream);
 
 /* Page score u_p = max over the group's query heads of
  * sum_c max(q_c kmin_c, q_c kmax_c) / sqrt(d) with the current query q; the

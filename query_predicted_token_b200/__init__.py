@@ -23,6 +23,7 @@ from ._lib import (  # noqa: F401
     make_event,
     predict_query,
     quest_build_meta,
+    quest_page_scores,
     quest_select,
     score_keys,
     select_topk,

@@ -61,6 +61,7 @@ SIGNATURES = {
     "asp_graph_destroy": (c_int, [c_void_p]),
     "asp_wait_selection": (c_int, [c_void_p, c_long]),
     "asp_quest_build_meta": (c_int, [POINTER(AspKv), c_int, c_void_p, c_void_p]),
+    "asp_quest_page_scores": (c_int, [c_void_p, c_int, c_int, POINTER(AspKv), c_void_p, c_int, c_void_p, c_void_p]),
     "asp_quest_select": (c_int, [c_void_p, c_int, c_int, POINTER(AspKv), c_void_p, c_int, c_int, c_void_p, c_void_p,
                                  c_void_p, c_void_p]),
     "asp_device_status": (c_int, [c_void_p, POINTER(c_int32)]),
@@ -210,6 +211,14 @@ def sparse_attend_noalloc(q: torch.Tensor, kv: KV, idx: Optional[torch.Tensor], 
 
 def quest_build_meta(kv: KV, quest_page: int, meta: torch.Tensor, stream=None) -> None:
     _check("asp_quest_build_meta", lib().asp_quest_build_meta(kv.ref, int(quest_page), _ptr(meta), _stream(stream)))
+
+
+def quest_page_scores(q: torch.Tensor, kv: KV, meta: torch.Tensor, quest_page: int, page_scores: torch.Tensor,
+                      stream=None) -> None:
+    """Page bounds of every page with the current query (the scan half of quest_select)."""
+    _check("asp_quest_page_scores", lib().asp_quest_page_scores(
+        q.data_ptr(), dtype_code(q), q.shape[1], kv.ref, meta.data_ptr(), int(quest_page),
+        page_scores.data_ptr(), _stream(stream)))
 
 
 def quest_select(q: torch.Tensor, kv: KV, meta: torch.Tensor, quest_page: int, C: int, page_scores: torch.Tensor,

@@ -432,17 +432,35 @@ asp_status asp_quest_build_meta(const asp_kv* kv, int quest_page, void* meta, as
   return cuda_status(asp::launch_quest_meta(view_of(kv), quest_page, meta, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-asp_status asp_quest_select(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv, const void* meta,
-                            int quest_page, int C, float* page_scores, int32_t* idx, int32_t* count,
-                            asp_stream_t stream) {
+namespace {
+asp_status check_quest(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv, const void* meta,
+                       int quest_page, float* page_scores) {
   asp_status st = check_kv(kv, false);
   if (st != ASP_OK) return st;
-  if (!q || !meta || !page_scores || !idx || !count || C <= 0 || quest_page <= 0) return ASP_ERR_INVALID_ARG;
+  if (!q || !meta || !page_scores || quest_page <= 0) return ASP_ERR_INVALID_ARG;
   if (q_dtype != ASP_F32 && q_dtype != ASP_BF16) return ASP_ERR_INVALID_ARG;
   if (n_q_heads <= 0 || n_q_heads % kv->n_kv_heads) return ASP_ERR_INVALID_ARG;
   if (!group_ok(n_q_heads, kv->n_kv_heads)) return ASP_ERR_UNSUPPORTED;
   if (quest_page % 16 || quest_page > 256) return ASP_ERR_UNSUPPORTED;
   if (kv->page_size && kv->page_size != quest_page) return ASP_ERR_UNSUPPORTED;
+  return ASP_OK;
+}
+}  // namespace
+
+asp_status asp_quest_page_scores(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv, const void* meta,
+                                 int quest_page, float* page_scores, asp_stream_t stream) {
+  asp_status st = check_quest(q, q_dtype, n_q_heads, kv, meta, quest_page, page_scores);
+  if (st != ASP_OK) return st;
+  return cuda_status(asp::launch_quest_score(q, q_dtype == ASP_F32, n_q_heads, view_of(kv), meta, quest_page,
+                                             page_scores, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+asp_status asp_quest_select(const void* q, asp_dtype q_dtype, int n_q_heads, const asp_kv* kv, const void* meta,
+                            int quest_page, int C, float* page_scores, int32_t* idx, int32_t* count,
+                            asp_stream_t stream) {
+  asp_status st = check_quest(q, q_dtype, n_q_heads, kv, meta, quest_page, page_scores);
+  if (st != ASP_OK) return st;
+  if (!idx || !count || C <= 0) return ASP_ERR_INVALID_ARG;
   if (!asp::select_supported(kv->t_max, quest_page)) return ASP_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = asp::launch_quest_score(q, q_dtype == ASP_F32, n_q_heads, view_of(kv), meta, quest_page,

@@ -54,6 +54,9 @@ struct AttParams {
   int n_items;   // units * splits: the persistent kernel's work items
   int lean;      // launch the kernel form with fewer registers
   int ctas;      // its grid
+  int tiles_per_unit;      // gather kernel: 16-row tiles planned per unit
+  long long total_tiles;   // gather kernel: units * tiles_per_unit
+  int stages;              // gather kernel: stages per producer / consumer pair
   float* part_o;
   float* part_ml;
   void* out;
@@ -728,6 +731,441 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
   }
 }
 
+// ---- bf16 cache and query: persistent gather, producer / consumer warp pairs --
+//
+// Every (sequence, KV head) unit is planned for C + max_tail rows, cut into
+// 16-row tiles; the flattened tiles of all units are split into equal
+// contiguous ranges, one per CTA (at most one CTA per SM), so every CTA gathers
+// the same number of rows whatever the split of units.  Within a CTA, tile k of
+// its range belongs to warp pair k % NP: producer warp NP + w issues the pair's
+// tiles into the pair's ring of SP stages (16 K + 16 V rows each, 16-byte padded
+// pitch for conflict-free ldmatrix) and consumer warp w consumes them in the same
+// order -- one in-order ring per pair, so no barrier phase can be waited on
+// before its predecessor completed.
+//   producer: walks its tiles with the unit and tile position kept incrementally
+//     (no division per tile), the unit's lengths cached; two tiles per round
+//     (lanes 0-15 and 16-31 resolve one row each); index loads two rounds ahead
+//     of the copies, page lookups one round ahead; the 32 rows of a tile go in
+//     as 16-byte cp.async (several rows per warp instruction, rows that are not
+//     read zero-filled), each lane's copies arriving on the stage's "full"
+//     barrier when they land, lane 0 adding the tile's row mask;
+//   consumer: the tensor-core logits, online softmax and P.V of
+//     attend_mma_kernel, then releases the stage on its "empty" barrier.
+// The rows a CTA holds of one unit form a segment: at a segment's end the
+// consumers merge through shared memory; a unit held by one CTA is written out
+// directly, otherwise the CTA writes a partial (max, sum, unnormalised output)
+// and attend_gather_merge_kernel combines them.  The producers run on into the
+// next segment meanwhile.  Every barrier wait is bounded (ASP_DEV_WAIT_LIMIT).
+constexpr int kGatherPairs = 6;
+constexpr int kGatherThreads = 2 * kGatherPairs * 32;
+
+// Tiles [t0, t1) of CTA c out of I over N CTAs; owner of tile i.
+__device__ __forceinline__ long long tile_start(long long c, long long I, long long N) { return c * I / N; }
+__device__ __forceinline__ long long tile_owner(long long i, long long I, long long N) { return ((i + 1) * N - 1) / I; }
+
+// Bounded wait that also gives up once another warp of the CTA has given up.
+__device__ __forceinline__ bool gather_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  for (uint32_t i = 0; i < kWaitTries; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+  }
+  flag_status(ASP_DEV_WAIT_LIMIT);
+  *abort_flag = 1;
+  return false;
+}
+
+__device__ __forceinline__ void consumers_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kGatherPairs * 32) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_plain(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kGatherThreads, 1) attend_gather_kernel(AttParams p) {
+  constexpr int NP = kGatherPairs;
+  constexpr int ROW_BYTES = D * 2;
+  constexpr int STRIDE = ROW_BYTES + 16;
+  constexpr int HALF = kTile * STRIDE;
+  constexpr int STAGE = 2 * HALF;
+  constexpr int KS = D / 16;
+  constexpr int NT = D / 8;
+  constexpr int CPR = ROW_BYTES / 16;   // 16-byte chunks per row
+  constexpr int RPI = 32 / CPR;         // rows per warp instruction
+  constexpr uint32_t kNone = 0xffffffffu;
+  static_assert(G >= 1 && G <= 8 && kTile == 16 && (32 % CPR) == 0, "layout");
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int SP = p.stages;   // stages per pair
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* const ring = smem;                                                 // [NP][SP] stages
+  float* const mo = reinterpret_cast<float*>(ring + (size_t)NP * SP * STAGE);   // [NP][G][D]
+  float* const mml = mo + NP * G * D;                                         // [NP][G][2]
+  uint64_t* const full = reinterpret_cast<uint64_t*>(mml + NP * G * 2);       // [NP][SP]
+  uint64_t* const empty = full + NP * SP;                                     // [NP][SP]
+  uint32_t* const masks = reinterpret_cast<uint32_t*>(empty + NP * SP);       // [NP][SP]
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(masks + NP * SP);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NP * SP; ++s) {
+      mbar_init(&full[s], 1);    // lane 0 of the producer; the copies add their own arrivals
+      mbar_init(&empty[s], 1);
+    }
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  __syncthreads();
+
+  const long long I = p.total_tiles, N = gridDim.x, c = blockIdx.x;
+  const long long t0 = tile_start(c, I, N), t1 = tile_start(c + 1, I, N);
+  if (t0 >= t1) return;
+  const int TPU = p.tiles_per_unit;
+  const int u_first = (int)(t0 / TPU);
+  const int nseg = (int)((t1 - 1) / TPU) - u_first + 1;
+  const int ntl = (int)(t1 - t0);
+  const int pair = warp % NP;
+  const int my_n = ntl > pair ? (ntl - pair + NP - 1) / NP : 0;   // the pair's tiles
+  uint8_t* const pring = ring + (size_t)pair * SP * STAGE;
+
+  if (warp >= NP) {
+    // ------------------------------------------------------------ producer
+    const int half = lane >> 4, rr = lane & 15;
+    // position of the pair's first tile; advanced by NP tiles per tile, by 2 NP per round
+    const long long gfirst = t0 + pair;
+    int unit0 = (int)(gfirst / TPU);
+    int tl0 = (int)(gfirst - (long long)unit0 * TPU);
+    // this lane's tile in round i is the pair's tile 2i + half
+    struct Pos {
+      int unit, tl;
+    };
+    auto step = [&](Pos q, int tiles) -> Pos {   // q moved on by tiles * NP CTA tiles
+      q.tl += tiles * NP;
+      while (q.tl >= TPU) {
+        q.tl -= TPU;
+        ++q.unit;
+      }
+      return q;
+    };
+    // the unit's lengths, reloaded only when the unit changes
+    int cu = -1, cT = 0, cn_sel = 0, ctb = 0, cn_rows = 0, cb = 0, ch = 0;
+    auto unit_params = [&](int unit) {
+      if (unit == cu) return;
+      cu = unit;
+      cb = unit / p.n_kv;
+      ch = unit - cb * p.n_kv;
+      int T = p.seq_lens ? __ldg(p.seq_lens + cb) : p.t_max;
+      cT = T < 0 ? 0 : (T > p.t_max ? p.t_max : T);
+      int n_sel = (p.C > 0 && p.count) ? __ldg(p.count + unit) : 0;
+      cn_sel = n_sel < 0 ? 0 : (n_sel > p.C ? p.C : n_sel);
+      int tb = cT;
+      if (p.tail_begin) {
+        tb = __ldg(p.tail_begin + cb);
+        tb = tb < 0 ? 0 : (tb > cT ? cT : tb);
+      }
+      ctb = tb;
+      int tail = cT - tb;
+      if (tail > p.max_tail) {
+        if (lane == 0 && pair == 0) flag_status(ASP_DEV_TAIL_LIMIT);
+        tail = p.max_tail;
+      }
+      cn_rows = cn_sel + tail;
+    };
+    // stage A: the raw index of this lane's row (loads issued, not waited for)
+    struct RowA {
+      int unit, r, raw;
+    };
+    auto stage_a = [&](Pos q, int j) -> RowA {
+      RowA a{-1, 0, 0};
+      if (j >= my_n) return a;
+      a.unit = q.unit;
+      a.r = q.tl * kTile + rr;
+      if (a.r < p.C) a.raw = __ldg(p.idx + (size_t)q.unit * p.C + a.r);
+      return a;
+    };
+    // stage B: the token (-1: not read) and, for a paged cache, its page (load issued)
+    struct RowB {
+      int unit, tok, page;
+    };
+    auto stage_b = [&](const RowA& a) -> RowB {
+      RowB bq{a.unit, -1, 0};
+      if (a.unit < 0) return bq;
+      unit_params(a.unit);
+      if (a.r >= cn_rows) return bq;
+      int tok;
+      if (a.r < cn_sel) {
+        tok = a.raw;
+        if (tok < 0 || tok >= cT) {
+          flag_status(ASP_DEV_BAD_INDEX);
+          return bq;
+        }
+        if (tok >= ctb) return bq;   // covered by the tail
+      } else {
+        tok = ctb + (a.r - cn_sel);
+      }
+      bq.tok = tok;
+      if (p.page_size) bq.page = __ldg(p.page_table + (size_t)cb * p.max_pages + tok / p.page_size);
+      return bq;
+    };
+    // stage C: the source row in the k / v arrays (32 bits: the cache fits in device memory)
+    auto stage_c = [&](const RowB& bq) -> uint32_t {
+      if (bq.tok < 0) return kNone;
+      if (p.page_size == 0) return (uint32_t)((size_t)bq.unit * p.t_max + bq.tok);
+      if (bq.page < 0 || bq.page >= p.n_pages) {
+        flag_status(ASP_DEV_BAD_PAGE);
+        return kNone;
+      }
+      const int h = bq.unit % p.n_kv;
+      return (uint32_t)(((size_t)bq.page * p.n_kv + h) * p.page_size + (bq.tok % p.page_size));
+    };
+
+    bool ok = true;
+    unit_params(unit0);               // its loads go out with the first index loads
+    Pos qA{unit0, tl0};               // position of this lane's tile in round 0
+    if (half) qA = step(qA, 1);
+    Pos qB = step(qA, 2), qC = step(qB, 2);
+    RowA aA = stage_a(qA, half), aB = stage_a(qB, 2 + half);
+    RowB bA = stage_b(aA);
+    const int rounds = (my_n + 1) / 2;
+#pragma unroll 1
+    for (int i = 0; i < rounds && ok; ++i) {
+      const RowA aC = stage_a(qC, 2 * (i + 2) + half);
+      const RowB bB = stage_b(aB);
+      const uint32_t row = stage_c(bA);
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int j = 2 * i + hf;   // the pair's tile
+        if (j >= my_n) break;
+        const int slot = j % SP;
+        if (j >= SP) {
+          ok = __all_sync(0xffffffffu, gather_wait(&empty[pair * SP + slot], (uint32_t)(j / SP - 1) & 1u, abort_flag));
+          if (!ok) break;
+        }
+        const uint32_t vm = (__ballot_sync(0xffffffffu, row != kNone) >> (16 * hf)) & 0xffffu;
+        if (vm) {
+          const uint32_t st = smem_u32(pring + (size_t)slot * STAGE);
+          const uint32_t c16 = (uint32_t)(lane % CPR) * 16u;
+#pragma unroll
+          for (int ins = 0; ins < 32 / RPI; ++ins) {
+            const int ri = RPI * ins + lane / CPR;   // 0-15 K rows, 16-31 V rows
+            const uint32_t src = __shfl_sync(0xffffffffu, row, 16 * hf + (ri & 15));
+            const bool valid = src != kNone;
+            const uint8_t* from = (ri < 16 ? p.k : p.v) + (valid ? (size_t)src * ROW_BYTES + c16 : 0);
+            const uint32_t dst = st + (uint32_t)((ri < 16 ? 0 : HALF) + (ri & 15) * STRIDE) + c16;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(from),
+                         "r"(valid ? 16 : 0)
+                         : "memory");
+          }
+          asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[pair * SP + slot]))
+                       : "memory");
+        }
+        __syncwarp();
+        if (lane == 0) {
+          masks[pair * SP + slot] = vm;
+          mbar_arrive_plain(&full[pair * SP + slot]);
+        }
+      }
+      qC = step(qC, 2);
+      aB = aC;
+      bA = bB;
+    }
+    if (!ok) asm volatile("cp.async.wait_all;" ::: "memory");   // let this producer's copies land
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int g = lane >> 2, t = lane & 3;
+  auto load_q = [&](int unit, uint32_t (&qa)[KS][2]) {
+    const int b = unit / p.n_kv, h = unit - b * p.n_kv;
+    const __nv_bfloat16* qrow =
+        static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.n_q_heads + h * G + (g < G ? g : 0)) * D;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      qa[kk][0] = g < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t)) : 0u;
+      qa[kk][1] = g < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 8 + 2 * t)) : 0u;
+    }
+  };
+  uint32_t qa[KS][2];
+  load_q(u_first, qa);
+  const int mat = lane >> 3, mrow = lane & 7;
+  const uint32_t k_off = (uint32_t)(((mat >> 1) * 8 + mrow) * STRIDE + (mat & 1) * 16);
+  const uint32_t v_off = (uint32_t)(HALF + ((mat & 1) * 8 + mrow) * STRIDE + (mat >> 1) * 16);
+  bool ok = true;
+  int j = 0;   // the pair's next tile
+  for (int sg = 0; sg < nseg; ++sg) {
+    const int u = u_first + sg;
+    const long long ua = (long long)u * TPU;
+    const long long hi = ua + TPU < t1 ? ua + TPU : t1;
+    // the pair's tiles before hi: CTA-local k = pair + NP * j < hi - t0
+    const long long khi = hi - t0 - pair;
+    const int jhi = khi > 0 ? (int)((khi + NP - 1) / NP) : 0;
+    float o[NT][2];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+#pragma unroll 1
+    for (; j < jhi && ok; ++j) {
+      const int slot = j % SP;
+      if (!__all_sync(0xffffffffu, gather_wait(&full[pair * SP + slot], (uint32_t)(j / SP) & 1u, abort_flag))) {
+        ok = false;
+        break;
+      }
+      const uint32_t vm = masks[pair * SP + slot];
+      if (vm) {
+        const uint32_t base = smem_u32(pring + (size_t)slot * STAGE);
+        float s0[2] = {0.f, 0.f}, s1[2] = {0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t kb[4];
+          ldsm_x4(kb, base + k_off + 32 * ks);
+          mma_top8(s0[0], s0[1], qa[ks][0], qa[ks][1], kb[0], kb[1]);
+          mma_top8(s1[0], s1[1], qa[ks][0], qa[ks][1], kb[2], kb[3]);
+        }
+        float x[4] = {s0[0] * p.qscale, s0[1] * p.qscale, s1[0] * p.qscale, s1[1] * p.qscale};
+        const int rows[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
+        float mloc = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (!((vm >> rows[e]) & 1u)) x[e] = -INFINITY;
+          mloc = fmaxf(mloc, x[e]);
+        }
+        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+        const float m_new = fmaxf(m_run, mloc);
+        const float corr = (m_new == -INFINITY) ? 1.f : ex2(m_run - m_new);
+        float pr[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pr[e] = (x[e] == -INFINITY) ? 0.f : ex2(x[e] - m_new);
+        l_run = l_run * corr + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
+        m_run = m_new;
+        uint32_t pa0, pa2, pl0, pl2;
+        split_bf16x2(pr[0], pr[1], pa0, pl0);
+        split_bf16x2(pr[2], pr[3], pa2, pl2);
+        if (corr != 1.f) {
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            o[n][0] *= corr;
+            o[n][1] *= corr;
+          }
+        }
+#pragma unroll
+        for (int jj = 0; jj < D / 16; ++jj) {
+          uint32_t vb[4];
+          ldsm_x4_trans(vb, base + v_off + 32 * jj);
+          mma_top8(o[2 * jj][0], o[2 * jj][1], pa0, pa2, vb[0], vb[1]);
+          mma_top8(o[2 * jj + 1][0], o[2 * jj + 1][1], pa0, pa2, vb[2], vb[3]);
+          mma_top8(o[2 * jj][0], o[2 * jj][1], pl0, pl2, vb[0], vb[1]);
+          mma_top8(o[2 * jj + 1][0], o[2 * jj + 1][1], pl0, pl2, vb[2], vb[3]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_plain(&empty[pair * SP + slot]);
+    }
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+
+    // merge the consumers; a unit held by this CTA alone is written out
+    if (g < G) {
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+        *reinterpret_cast<float2*>(mo + (warp * G + g) * D + n * 8 + 2 * t) = make_float2(o[n][0], o[n][1]);
+      if (t == 0) {
+        mml[(warp * G + g) * 2 + 0] = m_run;
+        mml[(warp * G + g) * 2 + 1] = l_run;
+      }
+    }
+    consumers_sync();
+    // the next segment's query loads while the partials are combined
+    if (sg + 1 < nseg) load_q(u + 1, qa);
+    const bool whole = tile_owner(ua, I, N) == tile_owner(ua + TPU - 1, I, N);
+    const int pslot = 2 * (int)c + (sg == 0 ? 0 : 1);
+    const int b = u / p.n_kv, h = u - b * p.n_kv;
+    for (int e = threadIdx.x; e < G * D; e += NP * 32) {
+      const int gg = e / D, cc = e - gg * D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NP; ++w) M = fmaxf(M, mml[(w * G + gg) * 2]);
+      float L = 0.f, O = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < NP; ++w) {
+          const float mw = mml[(w * G + gg) * 2];
+          if (mw == -INFINITY) continue;
+          const float f = ex2(mw - M);
+          L += mml[(w * G + gg) * 2 + 1] * f;
+          O += mo[(w * G + gg) * D + cc] * f;
+        }
+      }
+      if (whole) {
+        const size_t bh = (size_t)b * p.n_q_heads + h * G + gg;
+        static_cast<__nv_bfloat16*>(p.out)[bh * D + cc] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
+        if (cc == 0 && p.lse) p.lse[bh] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+      } else {
+        p.part_o[((size_t)pslot * G + gg) * D + cc] = O;
+        if (cc == 0) {
+          p.part_ml[((size_t)pslot * G + gg) * 2 + 0] = M;
+          p.part_ml[((size_t)pslot * G + gg) * 2 + 1] = L;
+        }
+      }
+    }
+    consumers_sync();
+  }
+}
+
+// Log-sum-exp merge of the units that several CTAs of attend_gather_kernel share:
+// block (c, g) merges head g of the unit whose first tile lies in CTA c's range
+// and whose last tile lies past it (at most one per CTA).  The partials are read
+// eight CTAs at a time with independent loads.
+template <int D, int G>
+__global__ void __launch_bounds__(D) attend_gather_merge_kernel(AttParams p, int n_ctas) {
+  const long long I = p.total_tiles, N = n_ctas, c = blockIdx.x;
+  const int gg = blockIdx.y, cc = threadIdx.x;
+  const int TPU = p.tiles_per_unit;
+  const long long t0 = tile_start(c, I, N), t1 = tile_start(c + 1, I, N);
+  if (t0 >= t1) return;
+  const int u = (int)((t1 - 1) / TPU);
+  const long long ua = (long long)u * TPU;
+  if (ua < t0 || ua + TPU <= t1) return;
+  pdl_wait();   // the partials come from the previous kernel
+  const long long c1 = tile_owner(ua + TPU - 1, I, N);
+  const int first_slot = (int)(2 * c + (u == (int)(t0 / TPU) ? 0 : 1));
+  float M = -INFINITY, L = 0.f, O = 0.f;
+  for (long long base = c; base <= c1; base += 8) {
+    float mv[8], lv[8], ov[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const long long cx = base + i;
+      // CTAs with an empty range (more CTAs than tiles) hold no partial
+      const bool in = cx <= c1 && tile_start(cx, I, N) < tile_start(cx + 1, I, N);
+      const int s = cx == c ? first_slot : (int)(2 * cx);
+      mv[i] = in ? p.part_ml[((size_t)s * G + gg) * 2] : -INFINITY;
+      lv[i] = in ? p.part_ml[((size_t)s * G + gg) * 2 + 1] : 0.f;
+      ov[i] = in ? p.part_o[((size_t)s * G + gg) * D + cc] : 0.f;
+    }
+    float Mn = M;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) Mn = fmaxf(Mn, mv[i]);
+    if (Mn == -INFINITY) continue;
+    if (M != -INFINITY) {
+      const float f = ex2(M - Mn);
+      L *= f;
+      O *= f;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (mv[i] == -INFINITY) continue;
+      const float f = ex2(mv[i] - Mn);
+      L += lv[i] * f;
+      O += ov[i] * f;
+    }
+    M = Mn;
+  }
+  const int b = u / p.n_kv, h = u - b * p.n_kv;
+  const size_t bh = (size_t)b * p.n_q_heads + h * G + gg;
+  static_cast<__nv_bfloat16*>(p.out)[bh * D + cc] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
+  if (cc == 0 && p.lse) p.lse[bh] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+}
+
 // Log-sum-exp merge of the split partials: one CTA of D threads per query head.
 template <typename KT, int D>
 __global__ void __launch_bounds__(D) attend_merge_kernel(const float* __restrict__ part_o,
@@ -811,13 +1249,41 @@ cudaError_t dispatch_g(int G, const AttParams& p, cudaStream_t s) {
 
 }  // namespace
 
-// Split plan: as many splits per KV head as fit in one wave of resident CTAs on
-// a 148-SM B200 (by default 3 CTAs per SM for G <= 4, 2 for G = 8, set by the
-// registers), each split a multiple of 64 rows (one 16-row tile per warp).  A
-// pure function of the sizes, so the workspace size is known without a device.
+// Split plan of the per-item kernels: as many splits per KV head as fit in one
+// wave of resident CTAs on a 148-SM B200 (by default 3 CTAs per SM for G <= 4, 2
+// for G = 8, set by the registers), each split a multiple of 64 rows (one 16-row
+// tile per warp).  The gather kernel's plan (stand-alone calls; the decode step
+// keeps the per-item kernel, whose CTA fits beside the key scan's): every unit
+// planned for C + max_tail rows, its tiles spread evenly over at most one CTA per
+// SM (and at least 8 tiles per CTA), partials in 2 slots per CTA when a unit is
+// shared.  A pure function of the sizes, so the workspace size (the larger of the
+// two kernels' needs: which one runs depends on the data types) is known without
+// a device.
+constexpr int kGatherCtasMax = 148;
+constexpr int kGatherMaxTail = 4096;   // longer tails (dense attention) keep one CTA per item
+// The gather kernel pays a fixed cost per launch (filling 24 stages per SM before
+// the first tile, the partials' merge) that the per-item kernel, three CTAs per SM
+// streaming from the first row, does not: it is chosen from this many 16-row tiles
+// per SM on (measured on the Qwen3 shapes: 55 tiles per SM slower, 110 even, 446 a
+// third faster).
+constexpr int kGatherMinTilesPerCta = 200;
+
+// Whether any unit of the gather partition (total tiles over n CTAs, tpu tiles per
+// unit) is shared by several CTAs: at most one unit starts in a CTA's range and
+// runs past it.
+static bool gather_has_shared(long long total, int tpu, int n) {
+  for (long long c = 0; c < n; ++c) {
+    const long long t0 = c * total / n, t1 = (c + 1) * total / n;
+    if (t0 >= t1) continue;
+    const long long ua = ((t1 - 1) / tpu) * tpu;
+    if (ua >= t0 && ua + tpu > t1) return true;
+  }
+  return false;
+}
+
 AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail,
                        int ctas_per_sm) {
-  AttendPlan pl{1, 64, 0, 1, ctas_per_sm > 0 ? 1 : 0};
+  AttendPlan pl{1, 64, 0, 1, ctas_per_sm > 0 ? 1 : 0, 0, 0, 0};
   const long rows = (long)C + (max_tail > 0 ? max_tail : 0);
   const long units = (long)batch * n_kv_heads;
   if (rows <= 0 || units <= 0 || n_kv_heads <= 0) return pl;
@@ -841,8 +1307,76 @@ AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, i
     const size_t ml = (size_t)batch * n_q_heads * pl.splits * 2 * 4;
     pl.workspace_bytes = ((o + 255) / 256) * 256 + ((ml + 255) / 256) * 256;
   }
+  const int mt = max_tail > 0 ? max_tail : 0;
+  if (ctas_per_sm == 0 && mt <= (C > kGatherMaxTail ? C : kGatherMaxTail)) {
+    pl.tiles_per_unit = (int)((rows + kTile - 1) / kTile);
+    const long long total = (long long)units * pl.tiles_per_unit;
+    const long long n = (total + 7) / 8;
+    pl.gather_ctas = (int)(n < kGatherCtasMax ? n : kGatherCtasMax);
+    pl.gather = total >= (long long)kGatherMinTilesPerCta * kGatherCtasMax ? 1 : 0;
+    if (pl.gather && gather_has_shared(total, pl.tiles_per_unit, pl.gather_ctas)) {
+      const size_t slots = 2 * (size_t)pl.gather_ctas * G;
+      const size_t ws = ((slots * head_dim * 4 + 255) / 256) * 256 + ((slots * 2 * 4 + 255) / 256) * 256;
+      if (ws > pl.workspace_bytes) pl.workspace_bytes = ws;
+    }
+  }
   return pl;
 }
+
+namespace {
+
+int max_smem_optin() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 232448;
+  if (cache[dev] <= 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess && n > 0)
+      cache[dev] = n;
+  }
+  return cache[dev] > 0 ? cache[dev] : 232448;
+}
+
+// Shared memory of the gather kernel: SP stages of 16 K + 16 V rows (16-byte
+// padded pitch) per producer / consumer pair, the consumers' merge area, the
+// stage barriers, masks and the abort flag.
+template <int D, int G>
+constexpr size_t gather_smem(int SP) {
+  return (size_t)kGatherPairs * SP * 2 * kTile * (D * 2 + 16) + (size_t)kGatherPairs * G * (D + 2) * 4 +
+         (size_t)kGatherPairs * SP * (8 + 8 + 4) + 16;
+}
+
+template <int D, int G>
+cudaError_t launch_gather(AttParams p, cudaStream_t s) {
+  // as many stages per pair as fit (at most 6, at least 2)
+  const size_t budget = (size_t)max_smem_optin();
+  int SP = 6;
+  while (SP > 2 && gather_smem<D, G>(SP) > budget) --SP;
+  if (gather_smem<D, G>(SP) > budget) return cudaErrorInvalidConfiguration;
+  p.stages = SP;
+  const size_t smem = gather_smem<D, G>(SP);
+  auto kern = attend_gather_kernel<D, G>;
+  if (prepare_kernel((const void*)kern, smem, kGatherThreads) < 1) return cudaErrorInvalidConfiguration;
+  int n = p.ctas;
+  if (n > sm_count()) n = sm_count();
+  cudaError_t e = launch_prio(kern, dim3(n), dim3(kGatherThreads), smem, s, p);
+  if (e != cudaSuccess) return e;
+  if (!gather_has_shared(p.total_tiles, p.tiles_per_unit, n)) return cudaSuccess;
+  return launch_pdl(attend_gather_merge_kernel<D, G>, dim3(n, G), dim3(D), 0, s, p, n);
+}
+
+template <int D>
+cudaError_t dispatch_gather(int G, const AttParams& p, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_gather<D, 1>(p, s);
+    case 2: return launch_gather<D, 2>(p, s);
+    case 4: return launch_gather<D, 4>(p, s);
+    case 8: return launch_gather<D, 8>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
 
 cudaError_t launch_attend(const void* q, int q_f32, int n_q_heads, const KvView& kv, const int32_t* idx,
                           const int32_t* count, int C, const int32_t* tail_begin, int max_tail, void* out,
@@ -871,7 +1405,17 @@ cudaError_t launch_attend(const void* q, int q_f32, int n_q_heads, const KvView&
   p.ctas = plan.ctas > 0 ? plan.ctas : 1;
   p.lean = plan.lean;
   p.rows_per_split = plan.rows_per_split;
-  if (plan.splits > 1) {
+  p.tiles_per_unit = plan.tiles_per_unit;
+  p.total_tiles = (long long)kv.batch * kv.n_kv * plan.tiles_per_unit;
+  p.stages = 0;
+  const bool gather = plan.gather && !kv.kv_f32 && !q_f32 && (reinterpret_cast<uintptr_t>(q) & 15) == 0;
+  if (gather) {
+    p.ctas = plan.gather_ctas > 0 ? plan.gather_ctas : 1;
+    const size_t slots = 2 * (size_t)p.ctas * (n_q_heads / kv.n_kv);
+    p.part_o = static_cast<float*>(workspace);
+    p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                         ((slots * kv.head_dim * 4 + 255) / 256) * 256);
+  } else if (plan.splits > 1) {
     const size_t o = (size_t)kv.batch * n_q_heads * plan.splits * kv.head_dim * 4;
     p.part_o = static_cast<float*>(workspace);
     p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ((o + 255) / 256) * 256);
@@ -883,6 +1427,7 @@ cudaError_t launch_attend(const void* q, int q_f32, int n_q_heads, const KvView&
   p.lse = lse;
   p.qscale = kLog2e / sqrtf((float)kv.head_dim);
   const int G = n_q_heads / kv.n_kv;
+  if (gather) return kv.head_dim == 64 ? dispatch_gather<64>(G, p, s) : dispatch_gather<128>(G, p, s);
   if (kv.kv_f32) return kv.head_dim == 64 ? dispatch_g<float, 64>(G, p, s) : dispatch_g<float, 128>(G, p, s);
   if (!q_f32) return kv.head_dim == 64 ? dispatch_mma<64>(G, p, s) : dispatch_mma<128>(G, p, s);
   return kv.head_dim == 64 ? dispatch_g<__nv_bfloat16, 64>(G, p, s) : dispatch_g<__nv_bfloat16, 128>(G, p, s);

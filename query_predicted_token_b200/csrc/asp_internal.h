@@ -152,6 +152,9 @@ struct AttendPlan {
   size_t workspace_bytes;
   int ctas;   // CTAs of the (persistent) tensor-core attention grid
   int lean;   // 1: the kernel form with fewer registers (one CTA per SM beside the key scan)
+  int gather;           // 1: bf16 cache and query go through attend_gather_kernel
+  int tiles_per_unit;   // gather: 16-row tiles planned per (sequence, KV head) unit
+  int gather_ctas;      // gather: CTAs (at most one per SM)
 };
 // ctas_per_sm: resident CTAs per SM the grid is sized for (0: as many as fit).
 AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail,

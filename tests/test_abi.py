@@ -140,10 +140,56 @@ def test_select_validation(lib):
     assert lib.asp_select_topk(FAKE, None, 70000, 1, 1024, 8, FAKE, FAKE, None) == L.ASP_ERR_UNSUPPORTED
 
 
+def _ceil256(n):
+    return -(-n // 256) * 256
+
+
+def _ring_ws(B, Hq, Hkv, d, C, max_tail):
+    # the gather kernel (batches of at least 200 16-row tiles per SM): every unit
+    # planned for C + max_tail rows in 16-row tiles,
+    # spread over at most 148 CTAs (at least 8 tiles each); when a unit is shared
+    # by several CTAs, two partial slots per CTA, each G heads of (fp32 output,
+    # max, sum)
+    units, G = B * Hkv, Hq // Hkv
+    tpu = -(-(C + max_tail) // 16)
+    tiles = units * tpu
+    if tiles < 200 * 148:          # smaller batches keep the per-item kernel
+        return 0
+    n = min(148, -(-tiles // 8))
+    shared = False    # some unit starts in a CTA's range and runs past it
+    for c in range(n):
+        t0, t1 = c * tiles // n, (c + 1) * tiles // n
+        ua = (t1 - 1) // tpu * tpu
+        shared |= t0 < t1 and ua >= t0 and ua + tpu > t1
+    if not shared:
+        return 0
+    slots = 2 * n * G
+    return _ceil256(slots * d * 4) + _ceil256(slots * 2 * 4)
+
+
+def _split_ws(B, Hq, Hkv, d, C, max_tail, ctas_per_sm):
+    # the per-item kernels: splits of a multiple of 64 rows filling one wave
+    units, G = B * Hkv, Hq // Hkv
+    target = 148 * (ctas_per_sm or (2 if G >= 8 else 3))
+    splits = max(1, target // units)
+    rows = C + max_tail
+    per = -(-(-(-rows // splits)) // 64) * 64
+    splits = -(-rows // per)
+    if splits == 1:
+        return 0
+    return _ceil256(B * Hq * splits * d * 4) + _ceil256(B * Hq * splits * 2 * 4)
+
+
 def test_attend_workspace_rules(lib):
     need = lib.asp_attend_workspace_bytes(8, 32, 8, 128, 2048, 0)
     assert need > 0 and need % 256 == 0
-    assert lib.asp_attend_workspace_bytes(1, 4, 2, 64, 64, 0) == 0       # one split: no workspace
+    # the larger of the two kernels' needs (the data types decide which one runs)
+    for args in [(8, 32, 8, 128, 2048, 0), (1, 4, 2, 64, 64, 0), (16, 64, 8, 128, 2048, 0), (64, 32, 8, 128, 2048, 1),
+                 (1, 8, 1, 128, 5000, 0), (3, 6, 2, 64, 37, 4), (64, 256, 8, 128, 1024, 3), (32, 256, 8, 128, 2048, 5)]:
+        assert lib.asp_attend_workspace_bytes(*args) == max(_ring_ws(*args), _split_ws(*args, 0)), args
+    assert lib.asp_attend_workspace_bytes(1, 2, 1, 128, 5, 0) == 0     # one tile in one CTA: nothing to merge
+    # dense attention (a tail longer than 4096 and than C) keeps the per-item kernel only
+    assert lib.asp_attend_workspace_bytes(8, 32, 8, 128, 0, 32768) == _split_ws(8, 32, 8, 128, 0, 32768, 0)
     assert lib.asp_attend_workspace_bytes(8, 32, 8, 96, 2048, 0) == 0    # unsupported head_dim
     assert lib.asp_attend_workspace_bytes(8, 32, 8, 128, 0, 0) == 0      # nothing to attend
     kv = _kv(batch=8, n_kv_heads=8, t_max=32768)
@@ -165,8 +211,7 @@ def test_decode_workspace_holds_the_partials_and_the_histogram(lib):
     # -> 2 splits of 1024 rows; partials (fp32 out + (max, sum) per head and split),
     # each 256-byte aligned, then the [64, 2048] int32 histogram
     B, Hq, Hkv, d, C = 8, 32, 8, 128, 2048
-    splits = 148 // (B * Hkv)
-    parts = -(-(B * Hq * splits * d * 4) // 256) * 256 + -(-(B * Hq * splits * 2 * 4) // 256) * 256
+    parts = _split_ws(B, Hq, Hkv, d, C, 0, 1)
     dec = lib.asp_decode_workspace_bytes(B, Hq, Hkv, d, C, 0)
     assert dec == parts + B * Hkv * 2048 * 4
     # fewer splits than the stand-alone attention's plan (3 CTAs per SM)
@@ -225,6 +270,15 @@ def test_quest_validation(lib):
     assert lib.asp_quest_build_meta(ctypes.byref(kvp), 16, FAKE, None) == L.ASP_ERR_UNSUPPORTED   # page mismatch
     assert lib.asp_quest_select(FAKE, L.ASP_BF16, 8, ctypes.byref(kv), FAKE, 16, 0, FAKE, FAKE, FAKE, None) == \
         L.ASP_ERR_INVALID_ARG
+    # the page scores alone: the same checks, less the selection's
+    score = lambda kv, q=FAKE, meta=FAKE, page=16, ps=FAKE, hq=8: lib.asp_quest_page_scores(
+        q, L.ASP_BF16, hq, ctypes.byref(kv), meta, page, ps, None)
+    assert score(kv, q=None) == L.ASP_ERR_INVALID_ARG
+    assert score(kv, meta=None) == L.ASP_ERR_INVALID_ARG
+    assert score(kv, ps=None) == L.ASP_ERR_INVALID_ARG
+    assert score(kv, page=24) == L.ASP_ERR_UNSUPPORTED
+    assert score(kv, hq=7) == L.ASP_ERR_INVALID_ARG
+    assert score(kvp) == L.ASP_ERR_UNSUPPORTED                      # bounds pages must be the cache's pages
 
 
 def test_product_path_fails_loudly_without_the_library(monkeypatch, tmp_path):

@@ -287,6 +287,69 @@ def test_sparse_attend_many_splits_and_tail(dtype):
     assert_lse_close(lse, ref_lse)
 
 
+def _lens(n, lo, hi, seed):
+    return [int(x) for x in np.random.default_rng(seed).integers(lo, hi + 1, n)]
+
+
+# B, Hkv, G, d, C, lens, page_size, tail: each at least 200 16-row tiles per SM (the
+# gather kernel's range): ragged counts below C with a tail; a paged ragged batch with
+# groups of 8; d = 64 with one query head per KV head
+_GATHER_CASES = [
+    (64, 8, 4, 128, 1024, _lens(64, 600, 1500, 1), 0, 3),
+    (32, 8, 8, 128, 2048, _lens(32, 1000, 3000, 2), 16, 5),
+    (16, 16, 1, 64, 1900, [2000] * 16, 0, 0),
+]
+
+
+@pytest.mark.parametrize("case", _GATHER_CASES, ids=["ragged_tail_G4", "paged_G8", "d64_G1"])
+def test_sparse_attend_gather_kernel(case):
+    """bf16 attention on batches large enough for the persistent gather kernel:
+    units split over CTA boundaries (partials merged by the log-sum-exp kernel) and
+    CTAs holding several units, against the oracle."""
+    B, Hkv, G, d, C, lens, page_size, tail = case
+    assert B * Hkv * -(-(C + tail) // 16) >= 200 * 148
+    T = max(lens)
+    kvd, kv = make_cache(B, Hkv, d, T, torch.bfloat16, lens, page_size, seed=B + C)
+    tb = [max(0, t - tail) for t in lens]
+    idx, cnt = random_selection(B, Hkv, C, tb, seed=C + G)
+    q = torch.randn(B, Hkv * G, d, generator=_gen(B * 7 + d)).to(torch.bfloat16).to(DEV)
+    out = torch.full((B, Hkv * G, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    lse = torch.full((B, Hkv * G), float("nan"), device=DEV)
+    ws = torch.empty(max(16, asp.attend_workspace_bytes(B, Hkv * G, Hkv, d, C, tail)), dtype=torch.uint8, device=DEV)
+    tail_begin = torch.tensor(tb, dtype=torch.int32, device=DEV) if tail else None
+    asp.sparse_attend(q, kv, idx.to(DEV), cnt.to(DEV), C, out, lse, tail_begin, tail, ws)
+    torch.cuda.synchronize()
+    keys, vals = host_sequences(kvd)
+    ref, ref_lse = oracle.sparse_attend(np64(q), [keys[b] for b in range(B)], [vals[b] for b in range(B)],
+                                        idx.numpy(), cnt.numpy(), tb if tail else None)
+    assert_out_close(out, ref, torch.bfloat16, f"gather {case[:5]}")
+    assert_lse_close(lse, ref_lse)
+
+
+def test_gather_kernel_flags_out_of_range_indices_and_skips_them():
+    B, Hkv, G, d, C, T = 64, 8, 2, 128, 1024, 1100
+    kvd, kv = make_cache(B, Hkv, d, T, torch.bfloat16, [T] * B, seed=5)
+    idx, cnt = random_selection(B, Hkv, C, [T] * B, seed=6)
+    bad = idx.clone()
+    bad[3, 2, 10] = T + 5          # past the sequence
+    bad[40, 7, 1000] = -3          # negative
+    q = torch.randn(B, Hkv * G, d, generator=_gen(7)).to(torch.bfloat16).to(DEV)
+    out = torch.empty(B, Hkv * G, d, dtype=torch.bfloat16, device=DEV)
+    ws = torch.empty(max(16, asp.attend_workspace_bytes(B, Hkv * G, Hkv, d, C)), dtype=torch.uint8, device=DEV)
+    assert asp.device_status() == 0
+    asp.sparse_attend(q, kv, bad.to(DEV), cnt.to(DEV), C, out, workspace=ws)
+    assert asp.device_status() & asp.ASP_DEV_BAD_INDEX
+    keys, vals = host_sequences(kvd)
+    keep = bad.numpy().copy()
+    cnt_ref = cnt.numpy().copy()
+    for (b, h, j) in ((3, 2, 10), (40, 7, 1000)):   # the oracle attends the rest of the set
+        row = [x for x in keep[b, h, :cnt_ref[b, h]] if 0 <= x < T]
+        keep[b, h, :len(row)] = row
+        cnt_ref[b, h] = len(row)
+    ref, _ = oracle.sparse_attend(np64(q), [keys[b] for b in range(B)], [vals[b] for b in range(B)], keep, cnt_ref)
+    assert_out_close(out, ref, torch.bfloat16)
+
+
 def test_dense_attention_through_the_tail():
     """count = 0 and tail_begin = 0 attends every token: full attention."""
     B, Hkv, G, d, T = 2, 2, 2, 64, 3000
@@ -381,7 +444,12 @@ def test_quest_path(dtype, d, G, page_size):
     idx = torch.empty(B, Hkv, cap, dtype=torch.int32, device=DEV)
     cnt = torch.empty(B, Hkv, dtype=torch.int32, device=DEV)
     asp.quest_select(q, kv, meta, P, C, ps, idx, cnt)
+    ps_alone = torch.full_like(ps, float("nan"))
+    asp.quest_page_scores(q, kv, meta, P, ps_alone)
     torch.cuda.synchronize()
+    for b in range(B):   # the page scores alone are the selection's own, bit for bit
+        n = (lens[b] + P - 1) // P
+        assert torch.equal(ps_alone[b, :, :n], ps[b, :, :n])
     keys, _ = host_sequences(kvd)
     for b in range(B):
         for h in range(Hkv):
