@@ -49,6 +49,9 @@ def parse():
     ap.add_argument("--layers", type=int, default=36,
                     help="also time a stack of this many layers (each with its own cache), steady-state period "
                          "(1: no stack)")
+    ap.add_argument("--profile", default=None, choices=["scan", "scan_cuda_cores", "attend", "page_scan"],
+                    help="only build the workload and launch this kernel --steps times (for ncu captures); "
+                         "prints no JSON line")
     ap.add_argument("--side-streams", type=int, default=1,
                     help="with --layers: side streams the layers' selection chains alternate over")
     return ap.parse_args()
@@ -571,26 +574,44 @@ def full_attention_record(wl, kvd, kv, q_dev, stream, flush, steps, peak):
             "note": "every cached token through the tail path of asp_sparse_attend; one launch after an L2 flush"}
 # ----------------------------------------------------------------------------- selection recall
 def recall_analysis(wl, kv, dev):
-    """Recall of the true next query's top-C set (untimed): the step's own
-    selection (predicted query), the same step with raw ridge coefficients, and
-    the current query reused one step late."""
+    """Selection quality on the synthetic queries (untimed).
+
+    recall: share of the true next query's top-C set that a selection keeps -- the
+    step's own selection (softmax-normalised coefficients, windows' predictions
+    averaged), the same step with raw coefficients, the same step with the pooled-
+    features reading of the averaging, and the current query reused one step late.
+    by_reading: the same recall when the KV head's set is formed from its group
+    under the other readings of the GQA aggregation (mean query, summed softmax
+    mass, one set per query head), for the predicted and the current query.
+    window_overlap: overlap of the top-C set of the last of 17 successive true
+    queries with the 16 before it (mean over them, and with their union)."""
     import torch
     import query_predicted_token_b200 as asp
     import synth
-    from query_predicted_token_b200.recall import recall_report
+    from query_predicted_token_b200.recall import reading_recall, recall_report, window_overlap
     qhist, q_next = synth.query_history(wl, steps=2)
     q_t = q_next[0].to(wl.torch_dtype()).to(dev)
     q_true = q_next[1].to(wl.torch_dtype()).to(dev)     # the model's next query, as attention sees it
     B, Hq, d, C = wl.batch, wl.n_q_heads, wl.head_dim, wl.C
-    chosen = {}
-    for name, coef in (("predicted", "softmax"), ("predicted_raw_coefficients", "raw")):
-        st = asp.DecodeState(kv, Hq, asp.PredCfg(wl.W, wl.windows, wl.lam, coef), C, qhist.to(dev).contiguous())
+    chosen, qpred = {}, None
+    for name, coef, pool in (("predicted", "softmax", "predictions"),
+                             ("predicted_raw_coefficients", "raw", "predictions"),
+                             ("predicted_pooled_features", "softmax", "features")):
+        st = asp.DecodeState(kv, Hq, asp.PredCfg(wl.W, wl.windows, wl.lam, coef, pool), C,
+                             qhist.to(dev).contiguous())
         out = torch.empty(B, Hq, d, dtype=wl.torch_dtype(), device=dev)
         st.step(q_t, out)
         torch.cuda.synchronize()
         chosen[name] = tuple(t.clone() for t in st.selection)
+        if name == "predicted":
+            qpred = st.qpred.clone()
     res = recall_report(kv, C, q_true, {"current_query": q_t}, chosen)
     res = {k: round(v, 4) for k, v in res.items()}
+    res["by_reading"] = {r: {k: round(v, 4) for k, v in m.items()}
+                         for r, m in reading_recall(kv, C, q_true, {"predicted": qpred, "current_query": q_t}).items()}
+    hist = [qhist[:, :, s].to(wl.torch_dtype()).to(dev) for s in range(qhist.shape[2])]
+    res["window_overlap"] = {k: (round(v, 4) if isinstance(v, float) else v)
+                             for k, v in window_overlap(kv, C, hist).items()}
     res["note"] = ("mean over (sequence, KV head) of |S & S_true| / |S_true|, S_true = top C with the true "
                    "next query; synthetic AR(1) queries (rho %.2f), so an analogue, not the pages' numbers" % wl.rho)
     return res
@@ -665,6 +686,52 @@ def multi_layer_period(wl, layers, tokens, dev, side_streams=1):
     return res
 
 
+# ----------------------------------------------------------------------------- profiling launches
+def profile_launches(args):
+    """Builds the workload and launches one kernel --steps times, an L2 flush before
+    each, for an ncu capture of that kernel alone (scan: the key scan as the library
+    picks it; scan_cuda_cores: the CUDA-core scan on the same keys; attend: the
+    sparse attention's stand-alone plan over a random selection; page_scan: the
+    page-bound scan of the page-level path)."""
+    import torch
+    import query_predicted_token_b200 as asp
+    import synth
+    dev = torch.device("cuda", 0)
+    wl = synth.workload(args.workload)
+    B, Hq, Hkv, d, C = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.C
+    kvd = synth.kv_cache(wl, dev)
+    kv = asp.KV(kvd["k"], kvd["v"], kvd["seq_lens"], kvd["page_table"], t_max=wl.t_max)
+    lens = kvd["seq_lens"].cpu().tolist()
+    tail = 1 if kvd["page_table"] is not None else 0
+    snap = [t - tail for t in lens]
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    qpred = synth.query_history(wl, 1)[1][0].to(dev).contiguous()
+    q = qpred.to(wl.torch_dtype())
+    scores = torch.empty(B, Hkv, wl.t_max, device=dev)
+    if args.profile == "attend":
+        idx, cnt = (x.to(dev) for x in synth.random_selection(B, Hkv, C, snap, seed=wl.seed + 99))
+        tb = torch.tensor(snap, dtype=torch.int32, device=dev) if tail else None
+        out = torch.empty(B, Hq, d, dtype=wl.torch_dtype(), device=dev)
+        ws = torch.empty(max(16, asp.attend_workspace_bytes(B, Hq, Hkv, d, C, tail)), dtype=torch.uint8, device=dev)
+        fn = lambda: asp.sparse_attend(q, kv, idx, cnt, C, out, None, tb, tail, ws)
+    elif args.profile == "page_scan":
+        meta = torch.empty(B, Hkv, math.ceil(wl.t_max / QUEST_PAGE), 2, d, dtype=wl.torch_dtype(), device=dev)
+        asp.quest_build_meta(kv, QUEST_PAGE, meta)
+        ps = torch.empty(B, Hkv, math.ceil(wl.t_max / QUEST_PAGE), device=dev)
+        fn = lambda: asp.quest_page_scores(q, kv, meta, QUEST_PAGE, ps)
+    elif args.profile == "scan_cuda_cores":
+        fn = lambda: asp.score_keys_cuda_cores(qpred, kv, scores)
+    else:
+        fn = lambda: asp.score_keys(qpred, kv, scores)
+    for _ in range(args.steps):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    assert asp.device_status() == 0
+    print(f"profile {args.profile} {wl.name}: {args.steps} launches", flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- GPU arm
 SUB_WORKLOADS = ("qwen3_32b_shaped_32k", "longcot_ragged_paged_b64")
 
@@ -673,6 +740,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile:
+        return profile_launches(args)
     import torch
     import query_predicted_token_b200 as asp
     import synth

@@ -48,7 +48,7 @@
 extern "C" {
 #endif
 
-#define ASP_ABI_VERSION 2
+#define ASP_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define ASP_API __attribute__((visibility("default")))
@@ -76,6 +76,15 @@ typedef enum { ASP_F32 = 0, ASP_BF16 = 1 } asp_dtype;
  * method's softmax normalisation; RAW keeps the coefficients). */
 typedef enum { ASP_COEF_SOFTMAX = 0, ASP_COEF_RAW = 1 } asp_coef_mode;
 
+/* What "multi-window average pooling" averages.  PREDICTIONS (the reading the
+ * library follows by default): one ridge fit per window on that window's lagged
+ * queries, the windows' predictions averaged.  FEATURES (the recorded
+ * alternative): each window w pools the history into one feature, the mean of the
+ * w most recent vectors; one ridge fit on the windows' features one step back
+ * gives a weight per window (normalised as `coef` says), applied to the current
+ * features. */
+typedef enum { ASP_POOL_PREDICTIONS = 0, ASP_POOL_FEATURES = 1 } asp_pool_mode;
+
 /* Device status word bits (asp_device_status). */
 #define ASP_DEV_BAD_INDEX  0x1   /* a selected index outside [0, T_b) was skipped */
 #define ASP_DEV_BAD_PAGE   0x2   /* a page-table entry outside [0, n_pages) was skipped */
@@ -83,6 +92,8 @@ typedef enum { ASP_COEF_SOFTMAX = 0, ASP_COEF_RAW = 1 } asp_coef_mode;
 #define ASP_DEV_TAIL_LIMIT 0x8   /* a tail longer than max_tail was truncated */
 #define ASP_DEV_SELECT     0x10  /* a selection output position past C was skipped (a first-digit
                                     histogram that does not match the scores) */
+#define ASP_DEV_NAN_SCORE  0x20  /* the selection read a NaN score: invalid input, the chosen set
+                                    is then unspecified (it never holds more than C tokens) */
 
 /* The KV cache of one layer.
  *   page_size == 0: k, v are [batch, n_kv_heads, t_max, head_dim] (contiguous).
@@ -115,6 +126,7 @@ typedef struct {
   int n_windows;
   float lambda;          /* ridge parameter, > 0, added to the Gram diagonal unscaled */
   asp_coef_mode coef;
+  asp_pool_mode pool;    /* ASP_POOL_PREDICTIONS unless comparing the readings */
 } asp_pred_cfg;
 
 /* ---------------------------------------------------------------------------
@@ -156,6 +168,14 @@ ASP_API asp_status asp_predict_query(float* qhist, int ring_start, const void* q
  * not 64/128, batch > 8192). */
 ASP_API asp_status asp_score_keys(const float* qpred, int n_q_heads, const asp_kv* kv, float* scores,
                           asp_stream_t stream);
+
+/* Step 2 on the CUDA cores whatever the key type: the scan asp_score_keys runs for
+ * fp32 keys and page sizes other than 16, and for bf16 keys the comparison of its
+ * tensor-core scan (same arguments, errors and results within the score tolerance;
+ * the tensor-core path replaced it for bf16 keys because it reaches the copy
+ * bandwidth where this one is bound by instruction issue). */
+ASP_API asp_status asp_score_keys_cuda_cores(const float* qpred, int n_q_heads, const asp_kv* kv, float* scores,
+                                             asp_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Step 3 -- top-C token selection.
@@ -361,6 +381,15 @@ ASP_API asp_status asp_quest_select(const void* q, asp_dtype q_dtype, int n_q_he
 
 /* ---------------------------------------------------------------------------
  * Utilities. */
+
+/* Check of the device-side failure detection (no counterpart in the pages).  One
+ * warp waits on a shared-memory barrier that nothing arrives on, with the bounded
+ * wait every kernel of the library uses cut to `tries` attempts (each at most about
+ * 1 us); it gives up, records ASP_DEV_WAIT_LIMIT (read it with asp_device_status)
+ * and writes 1 to *returned (device int32) before it exits -- 2 would mean the wait
+ * succeeded.  No fault, trap or hang is involved.  Errors: ASP_ERR_INVALID_ARG
+ * (returned NULL, tries outside [1, 2^20]). */
+ASP_API asp_status asp_check_wait_limit(int tries, int32_t* returned, asp_stream_t stream);
 
 /* Reads and clears the device status word (ASP_DEV_* bits) after synchronising
  * `stream`.  Returns ASP_ERR_DEVICE when a bit was set, else ASP_OK/ASP_ERR_CUDA. */

@@ -27,3 +27,5 @@ from .attend import attend_set, sparse_attend  # noqa: F401
 from .quest import quest_meta, quest_page_scores, quest_select_row, quest_select  # noqa: F401
 from .flops import decode_flops, QWEN3_8B, QWEN3_32B  # noqa: F401
 from .pipeline import decode_step  # noqa: F401
+from .readings import (score_row_mean, score_row_mass, select_per_head, pooled_features,  # noqa: F401
+                       pooled_prediction, predict_query_pooled, set_overlap, recent_window_overlap)

@@ -8,6 +8,7 @@ from ._lib import (  # noqa: F401
     ASP_F32,
     ASP_DEV_BAD_INDEX,
     ASP_DEV_BAD_PAGE,
+    ASP_DEV_NAN_SCORE,
     ASP_DEV_SELECT,
     ASP_DEV_TAIL_LIMIT,
     ASP_DEV_WAIT_LIMIT,
@@ -17,6 +18,7 @@ from ._lib import (  # noqa: F401
     KV,
     PredCfg,
     attend_workspace_bytes,
+    check_wait_limit,
     device_status,
     event_handle,
     lib,
@@ -26,6 +28,7 @@ from ._lib import (  # noqa: F401
     quest_page_scores,
     quest_select,
     score_keys,
+    score_keys_cuda_cores,
     select_topk,
     sparse_attend,
     status_string,

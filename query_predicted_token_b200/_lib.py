@@ -19,7 +19,9 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libasp.so")
 ASP_OK, ASP_ERR_INVALID_ARG, ASP_ERR_UNSUPPORTED, ASP_ERR_WORKSPACE, ASP_ERR_CUDA, ASP_ERR_TIMEOUT, ASP_ERR_DEVICE = range(7)
 ASP_F32, ASP_BF16 = 0, 1
 ASP_COEF_SOFTMAX, ASP_COEF_RAW = 0, 1
+ASP_POOL_PREDICTIONS, ASP_POOL_FEATURES = 0, 1
 ASP_DEV_BAD_INDEX, ASP_DEV_BAD_PAGE, ASP_DEV_WAIT_LIMIT, ASP_DEV_TAIL_LIMIT, ASP_DEV_SELECT = 1, 2, 4, 8, 16
+ASP_DEV_NAN_SCORE = 32
 
 # every entry point of include/asp.h with its ctypes signature
 class AspKv(ctypes.Structure):
@@ -29,7 +31,8 @@ class AspKv(ctypes.Structure):
 
 
 class AspPredCfg(ctypes.Structure):
-    _fields_ = [("W", c_int), ("windows", POINTER(c_int)), ("n_windows", c_int), ("lam", c_float), ("coef", c_int)]
+    _fields_ = [("W", c_int), ("windows", POINTER(c_int)), ("n_windows", c_int), ("lam", c_float), ("coef", c_int),
+                ("pool", c_int)]
 
 
 class AspDecodeArgs(ctypes.Structure):
@@ -61,9 +64,11 @@ SIGNATURES = {
     "asp_graph_destroy": (c_int, [c_void_p]),
     "asp_wait_selection": (c_int, [c_void_p, c_long]),
     "asp_quest_build_meta": (c_int, [POINTER(AspKv), c_int, c_void_p, c_void_p]),
+    "asp_score_keys_cuda_cores": (c_int, [c_void_p, c_int, POINTER(AspKv), c_void_p, c_void_p]),
     "asp_quest_page_scores": (c_int, [c_void_p, c_int, c_int, POINTER(AspKv), c_void_p, c_int, c_void_p, c_void_p]),
     "asp_quest_select": (c_int, [c_void_p, c_int, c_int, POINTER(AspKv), c_void_p, c_int, c_int, c_void_p, c_void_p,
                                  c_void_p, c_void_p]),
+    "asp_check_wait_limit": (c_int, [c_int, c_void_p, c_void_p]),
     "asp_device_status": (c_int, [c_void_p, POINTER(c_int32)]),
     "asp_status_string": (ctypes.c_char_p, [c_int]),
     "asp_abi_version": (c_int, []),
@@ -155,10 +160,18 @@ class KV:
 
 
 class PredCfg:
-    def __init__(self, W: int, windows: Sequence[int], lam: float, coef: str = "softmax"):
+    """Predictor configuration.  ``coef``: "softmax" (the method's normalisation) or
+    "raw"; ``pool``: "predictions" (average the windows' predictions, the default
+    reading) or "features" (regress on the windows' pooled features)."""
+
+    def __init__(self, W: int, windows: Sequence[int], lam: float, coef: str = "softmax",
+                 pool: str = "predictions"):
+        if coef not in ("softmax", "raw") or pool not in ("predictions", "features"):
+            raise ValueError(f"coef {coef!r}, pool {pool!r}")
         self._win = (c_int * len(windows))(*[int(w) for w in windows])
         self.struct = AspPredCfg(int(W), ctypes.cast(self._win, POINTER(c_int)), len(windows), float(lam),
-                                 ASP_COEF_RAW if coef == "raw" else ASP_COEF_SOFTMAX)
+                                 ASP_COEF_RAW if coef == "raw" else ASP_COEF_SOFTMAX,
+                                 ASP_POOL_FEATURES if pool == "features" else ASP_POOL_PREDICTIONS)
         self.W = int(W)
 
     @property
@@ -176,6 +189,12 @@ def predict_query(qhist: torch.Tensor, ring_start: int, cfg: PredCfg, qpred: tor
 
 def score_keys(qpred: torch.Tensor, kv: KV, scores: torch.Tensor, stream=None) -> None:
     _check("asp_score_keys", lib().asp_score_keys(_ptr(qpred), qpred.shape[1], kv.ref, _ptr(scores), _stream(stream)))
+
+
+def score_keys_cuda_cores(qpred: torch.Tensor, kv: KV, scores: torch.Tensor, stream=None) -> None:
+    """The key scan on the CUDA cores (the tensor-core scan's comparison for bf16 keys)."""
+    _check("asp_score_keys_cuda_cores", lib().asp_score_keys_cuda_cores(
+        qpred.data_ptr(), qpred.shape[1], kv.ref, scores.data_ptr(), _stream(stream)))
 
 
 def select_topk(scores: torch.Tensor, seq_lens: Optional[torch.Tensor], C: int, idx: torch.Tensor,
@@ -235,6 +254,11 @@ def append_kv(kv: KV, k_new: torch.Tensor, v_new: torch.Tensor, tail_begin: Opti
     old lengths; ``quest_meta`` (page bounds) is kept current."""
     _check("asp_append_kv", lib().asp_append_kv(kv.ref, _ptr(k_new), _ptr(v_new), _ptr(tail_begin),
                                                 _ptr(quest_meta), int(quest_page), _stream(stream)))
+
+
+def check_wait_limit(tries: int, returned: torch.Tensor, stream=None) -> None:
+    """Runs the bounded-wait check (see asp.h): ``returned`` int32 [1] gets 1 when the wait gave up."""
+    _check("asp_check_wait_limit", lib().asp_check_wait_limit(int(tries), returned.data_ptr(), _stream(stream)))
 
 
 def device_status(stream=None) -> int:

@@ -114,6 +114,7 @@ asp_status check_pred(const asp_pred_cfg* cfg, int ring_start) {
     if (cfg->windows[i] < 1 || cfg->windows[i] > cfg->W) return ASP_ERR_INVALID_ARG;
   if (!(cfg->lambda > 0.0f) || !std::isfinite(cfg->lambda)) return ASP_ERR_INVALID_ARG;
   if (cfg->coef != ASP_COEF_SOFTMAX && cfg->coef != ASP_COEF_RAW) return ASP_ERR_INVALID_ARG;
+  if (cfg->pool != ASP_POOL_PREDICTIONS && cfg->pool != ASP_POOL_FEATURES) return ASP_ERR_INVALID_ARG;
   if (ring_start < 0 || ring_start > cfg->W) return ASP_ERR_INVALID_ARG;
   return ASP_OK;
 }
@@ -153,6 +154,7 @@ asp::PredictArgs predict_args(float* qhist, int ring_start, const void* q_new, a
   }
   a.lam = (double)cfg->lambda;
   a.coef_raw = cfg->coef == ASP_COEF_RAW;
+  a.pool_features = cfg->pool == ASP_POOL_FEATURES;
   a.qpred = qpred;
   return a;
 }
@@ -231,6 +233,18 @@ asp_status asp_score_keys(const float* qpred, int n_q_heads, const asp_kv* kv, f
   if (!group_ok(n_q_heads, kv->n_kv_heads)) return ASP_ERR_UNSUPPORTED;
   if (kv->batch > kMaxScoreBatch) return ASP_ERR_UNSUPPORTED;
   return cuda_status(asp::launch_score(qpred, n_q_heads, view_of(kv), scores, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+asp_status asp_score_keys_cuda_cores(const float* qpred, int n_q_heads, const asp_kv* kv, float* scores,
+                                     asp_stream_t stream) {
+  asp_status st = check_kv(kv, false);
+  if (st != ASP_OK) return st;
+  if (!qpred || !scores) return ASP_ERR_INVALID_ARG;
+  if (n_q_heads <= 0 || n_q_heads % kv->n_kv_heads) return ASP_ERR_INVALID_ARG;
+  if (!group_ok(n_q_heads, kv->n_kv_heads)) return ASP_ERR_UNSUPPORTED;
+  if (kv->batch > kMaxScoreBatch) return ASP_ERR_UNSUPPORTED;
+  return cuda_status(asp::launch_score_cuda_cores(qpred, n_q_heads, view_of(kv), scores,
+                                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
 asp_status asp_select_topk(const float* scores, const int32_t* seq_lens, int batch, int n_kv_heads, int t_max, int C,
@@ -479,6 +493,11 @@ asp_status asp_quest_select(const void* q, asp_dtype q_dtype, int n_q_heads, con
   sa.count = count;
   sa.hist0 = nullptr;
   return cuda_status(asp::launch_select(sa, s));
+}
+
+asp_status asp_check_wait_limit(int tries, int32_t* returned, asp_stream_t stream) {
+  if (!returned || tries < 1 || tries > (1 << 20)) return ASP_ERR_INVALID_ARG;
+  return cuda_status(asp::launch_wait_limit_check(tries, returned, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 asp_status asp_device_status(asp_stream_t stream, int32_t* bits_out) {

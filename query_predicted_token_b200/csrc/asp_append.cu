@@ -102,6 +102,27 @@ cudaError_t launch_append(const KvView& kv, const void* k_new, const void* v_new
              : append_t<__nv_bfloat16, 128>(kv, k_new, v_new, seq_lens, tail_begin, meta, quest_page, s);
 }
 
+namespace {
+// One warp waits on a shared-memory barrier that nothing arrives on, with the
+// library's bounded wait cut to `tries` attempts; it must give up, record
+// ASP_DEV_WAIT_LIMIT and return, which *returned = 1 shows.
+__global__ void wait_limit_kernel(uint32_t tries, int32_t* returned) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+  const bool ok = __all_sync(0xffffffffu, mbar_wait_n(&bar, 0u, tries));
+  if (threadIdx.x == 0) *returned = ok ? 2 : 1;
+}
+}  // namespace
+
+cudaError_t launch_wait_limit_check(int tries, int32_t* returned, cudaStream_t s) {
+  wait_limit_kernel<<<1, 32, 0, s>>>((uint32_t)tries, returned);
+  return cudaGetLastError();
+}
+
 ASP_STATUS_READER(read_status_append)
 
 }  // namespace asp

@@ -74,11 +74,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait: about 2^20 tries of at most ~1 us each, i.e. at most ~1 s.
 constexpr uint32_t kWaitTries = 1u << 20;
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitTries; ++i)
+// Waits for the barrier phase of `parity`, giving up after `tries` attempts: then
+// ASP_DEV_WAIT_LIMIT is recorded and false returned.
+__device__ __forceinline__ bool mbar_wait_n(uint64_t* bar, uint32_t parity, uint32_t tries) {
+  for (uint32_t i = 0; i < tries; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   flag_status(ASP_DEV_WAIT_LIMIT);
   return false;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_n(bar, parity, kWaitTries);
 }
 
 // Orders earlier generic-proxy accesses of shared memory before later

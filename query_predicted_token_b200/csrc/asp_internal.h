@@ -86,6 +86,7 @@ struct PredictArgs {
   int wmax;
   double lam;
   int coef_raw;
+  int pool_features;      // 1: regress on the windows' pooled features (the recorded alternative reading)
   float* qpred;
   int win_fast;           // set by launch_predict: windows sorted, powers of two, one round of lanes
 };
@@ -114,6 +115,11 @@ cudaError_t launch_append(const KvView& kv, const void* k_new, const void* v_new
 // starts streaming keys before that kernel has finished.
 cudaError_t launch_score(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s,
                          int32_t* hist = nullptr, bool early = false);
+
+// The key scan on the CUDA cores whatever the key type (the path of fp32 keys and
+// other page sizes; for bf16 keys the comparison of the tensor-core scan).
+cudaError_t launch_score_cuda_cores(const float* qpred, int n_q_heads, const KvView& kv, float* scores,
+                                    cudaStream_t s, int32_t* hist = nullptr);
 
 // Tensor-core key scan (bf16 keys, head_dim 64/128, contiguous or 16-token pages,
 // G in {1,2,4,8}, 16-byte aligned qpred); launch_score uses it when supported.
@@ -168,6 +174,11 @@ cudaError_t launch_attend(const void* q, int q_f32, int n_q_heads, const KvView&
 cudaError_t launch_attend_noalloc(const void* q, int q_f32, int n_q_heads, const KvView& kv, const int32_t* idx,
                                   const int32_t* count, int C, const int32_t* tail_begin, int max_tail, void* out,
                                   float* lse, const AttendPlan& plan, cudaStream_t s);
+
+// ---- failure detection ----------------------------------------------------------
+// One warp waits on a barrier nothing arrives on, bounded to `tries` attempts;
+// *returned = 1 once it has given up (2 if the wait had succeeded).
+cudaError_t launch_wait_limit_check(int tries, int32_t* returned, cudaStream_t s);
 
 // ---- comparison path ----------------------------------------------------------
 cudaError_t launch_quest_meta(const KvView& kv, int quest_page, void* meta, cudaStream_t s);

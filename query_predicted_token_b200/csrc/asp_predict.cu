@@ -367,8 +367,155 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
 }
 
 
+// ---- the recorded alternative reading of the pooling: regress on pooled features ----
+//
+// One warp per query head.  With h[v] = q_{t-v} (v = 0: the target q_t), window
+// w's feature is the mean of its w most recent vectors, f_w(t) = mean(h[0..w-1]),
+// and one step back f_w(t-1) = mean(h[1..w]).  The ridge fit of q_t on the
+// features f_w(t-1) (samples = channels) is a k x k system (k windows, at most
+// 8): the features are formed in fp64 in shared memory (each lane its own
+// channels), the Gram and right-hand side reduced over the warp in fp64 and solved
+// by lane 0 (Cholesky, fp64); the weights (softmax or raw) apply to f_w(t).
+constexpr int kPoolMax = 8;
+
+template <int D, int NV>
+__global__ void __launch_bounds__(kWarps * 32) predict_pooled_kernel(PredictArgs a) {
+  constexpr int CPL = D / 32;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int head = blockIdx.x * kWarps + warp;
+  pdl_trigger();
+  if (a.zero) {   // clear the next kernel's histogram, as predict_kernel does
+    const size_t n4 = a.zero_words / 4;
+    int4* z4 = reinterpret_cast<int4*>(a.zero);
+    for (size_t i = (size_t)head * 32 + lane; i < n4; i += (size_t)gridDim.x * kWarps * 32) z4[i] = make_int4(0, 0, 0, 0);
+    for (size_t i = n4 * 4 + (size_t)head * 32 + lane; i < a.zero_words; i += (size_t)gridDim.x * kWarps * 32) a.zero[i] = 0;
+  }
+  if (head >= a.n_heads) return;
+  // per warp: features [2][kPoolMax][D] (cur, prev), then the k x k Gram and rhs
+  double* feat = reinterpret_cast<double*>(smem) + (size_t)warp * (2 * kPoolMax * D + kPoolMax * (kPoolMax + 1));
+  double* G = feat + 2 * kPoolMax * D;
+  double* rhs = G + kPoolMax * kPoolMax;
+  const int k = a.n_win;
+  const int n = a.wmax + 1;
+  const int nslot = a.W + 1;
+  float* hist = a.qhist + (size_t)head * nslot * D;
+  const int start = a.q_new ? a.ring_start + 1 : a.ring_start;
+  float h[NV][CPL];
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) h[v][c] = 0.f;
+    if (v < n) {
+      int slot = start + a.W - v;
+      if (slot >= nslot) slot -= nslot;
+      if (v == 0 && a.q_new) {
+        const size_t off = (size_t)head * D + lane * CPL;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c)
+          h[0][c] = a.q_new_f32 ? static_cast<const float*>(a.q_new)[off + c]
+                                : __bfloat162float(static_cast<const __nv_bfloat16*>(a.q_new)[off + c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) h[v][c] = hist[(size_t)slot * D + lane * CPL + c];
+      }
+    }
+  }
+  if (a.q_new) {   // push q_t into the ring: it replaces the oldest slot (ring_start)
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) hist[(size_t)a.ring_start * D + lane * CPL + c] = h[0][c];
+  }
+  // features of this lane's channels
+  for (int i = 0; i < k; ++i) {
+    const int w = a.windows[i];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      double cur = 0.0, prev = 0.0;
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        if (v < w) cur += (double)h[v][c];
+        if (v >= 1 && v <= w) prev += (double)h[v][c];
+      }
+      feat[(size_t)i * D + lane * CPL + c] = cur / w;
+      feat[(size_t)(kPoolMax + i) * D + lane * CPL + c] = prev / w;
+    }
+  }
+  __syncwarp();
+  // Gram of the one-step-back features and the right-hand side, reduced over the warp
+  for (int i = 0; i < k; ++i) {
+    for (int j = 0; j <= i; ++j) {
+      double part = 0.0;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c)
+        part += feat[(size_t)(kPoolMax + i) * D + lane * CPL + c] * feat[(size_t)(kPoolMax + j) * D + lane * CPL + c];
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      if (lane == 0) G[i * kPoolMax + j] = part + (i == j ? a.lam : 0.0);
+    }
+    double part = 0.0;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) part += feat[(size_t)(kPoolMax + i) * D + lane * CPL + c] * (double)h[0][c];
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) rhs[i] = part;
+  }
+  __syncwarp();
+  if (lane == 0) {
+    // Cholesky G = L L^T (lower triangle in place), then L z = rhs, L^T beta = z
+    for (int j = 0; j < k; ++j) {
+      double d = G[j * kPoolMax + j];
+      for (int m = 0; m < j; ++m) d -= G[j * kPoolMax + m] * G[j * kPoolMax + m];
+      const double ljj = sqrt(d);
+      G[j * kPoolMax + j] = ljj;
+      for (int i = j + 1; i < k; ++i) {
+        double e = G[i * kPoolMax + j];
+        for (int m = 0; m < j; ++m) e -= G[i * kPoolMax + m] * G[j * kPoolMax + m];
+        G[i * kPoolMax + j] = e / ljj;
+      }
+    }
+    for (int i = 0; i < k; ++i) {
+      double e = rhs[i];
+      for (int m = 0; m < i; ++m) e -= G[i * kPoolMax + m] * rhs[m];
+      rhs[i] = e / G[i * kPoolMax + i];
+    }
+    for (int i = k - 1; i >= 0; --i) {
+      double e = rhs[i];
+      for (int m = i + 1; m < k; ++m) e -= G[m * kPoolMax + i] * rhs[m];
+      rhs[i] = e / G[i * kPoolMax + i];
+    }
+    if (!a.coef_raw) {   // softmax over the k coefficients
+      double mx = rhs[0];
+      for (int i = 1; i < k; ++i) mx = fmax(mx, rhs[i]);
+      double sum = 0.0;
+      for (int i = 0; i < k; ++i) {
+        rhs[i] = exp(rhs[i] - mx);
+        sum += rhs[i];
+      }
+      for (int i = 0; i < k; ++i) rhs[i] /= sum;
+    }
+  }
+  __syncwarp();
+  float* out = a.qpred + (size_t)head * D + lane * CPL;
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) {
+    double acc = 0.0;
+    for (int i = 0; i < k; ++i) acc += rhs[i] * feat[(size_t)i * D + lane * CPL + c];
+    out[c] = (float)acc;
+  }
+}
+
+template <int D, int NV>
+cudaError_t launch_pooled_t(const PredictArgs& a, cudaStream_t s) {
+  const int grid = (a.n_heads + kWarps - 1) / kWarps;
+  const size_t smem = (size_t)kWarps * (2 * kPoolMax * D + kPoolMax * (kPoolMax + 1)) * sizeof(double);
+  auto kern = predict_pooled_kernel<D, NV>;
+  if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
+  return launch_prio(kern, dim3(grid), dim3(kWarps * 32), smem, s, a);
+}
+
 template <int D, int NV>
 cudaError_t launch_t(const PredictArgs& a, cudaStream_t s) {
+  if (a.pool_features) return launch_pooled_t<D, NV>(a, s);
   const int grid = (a.n_heads + kWarps - 1) / kWarps;
   const size_t smem = kWarps * Solve<NV>::kBytes;
   const bool exact = a.wmax == NV - 1;

@@ -279,6 +279,11 @@ cudaError_t dispatch_g(int G, const ScoreParams& p, cudaStream_t s) {
 cudaError_t launch_score(const float* qpred, int n_q_heads, const KvView& kv, float* scores, cudaStream_t s,
                          int32_t* hist, bool early) {
   if (score_tc_supported(kv, n_q_heads, qpred)) return launch_score_tc(qpred, n_q_heads, kv, scores, s, hist, early);
+  return launch_score_cuda_cores(qpred, n_q_heads, kv, scores, s, hist);
+}
+
+cudaError_t launch_score_cuda_cores(const float* qpred, int n_q_heads, const KvView& kv, float* scores,
+                                    cudaStream_t s, int32_t* hist) {
   ScoreParams p;
   p.qpred = qpred;
   p.n_q_heads = n_q_heads;

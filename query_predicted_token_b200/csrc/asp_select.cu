@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   // With the first histogram given, the threshold digit is found while the row's
   // scores load, and the units are classified and packed straight from registers.
   const bool fused = FUSED;
+  bool nan_seen = false;   // a NaN score (invalid input) in the part of the row this thread read
   if (FUSED && !(!own_h0 && vec && a.key_cap >= kWarps * 4)) {   // the launch rule was not met
     if (tid == 0) flag_status(ASP_DEV_SELECT);
     return;
@@ -129,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
       for (int u = 0; u < U; ++u) {
         const int i4 = base + u * kThreads + tid;
         const uint32_t k4[4] = {order_key(f[u].x), order_key(f[u].y), order_key(f[u].z), order_key(f[u].w)};
+        nan_seen |= i4 < n4 && (isnan(f[u].x) || isnan(f[u].y) || isnan(f[u].z) || isnan(f[u].w));
         if (i4 < n4) *reinterpret_cast<uint4*>(&keys[4 * i4]) = make_uint4(k4[0], k4[1], k4[2], k4[3]);
         if (own_h0) {
 #pragma unroll
@@ -141,13 +143,15 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
       const int i = base + tid;
       uint32_t key = 0u;
       if (i < n) {
-        key = order_key(srow[i]);
+        const float sv = srow[i];
+        nan_seen |= isnan(sv);
+        key = order_key(sv);
         if (cached) keys[i] = key;
       }
       if (own_h0) count_digit(h0, i < n, key >> kTopShift);
     }
   }
-  if (!fused) __syncthreads();
+  if (!fused && __syncthreads_or(nan_seen) && tid == 0) flag_status(ASP_DEV_NAN_SCORE);
 
   // Finds the digit (of width nb) that holds the krem-th largest of the counted
   // keys, given this CTA's histogram h (or the row's global one).
@@ -274,6 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
         for (int c = 0; c < 4; ++c) {
           sv[c] = i + c < w1 && fv[c] >= lo_f;
           gt[c] = fv[c] >= hi_f;
+          nan_seen |= i + c < w1 && isnan(fv[c]);
         }
         // rank of unit (lane, c) among the chunk's survivors: all of the lower
         // lanes' survivors, then this lane's earlier ones
@@ -296,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
         n_packed += total;
       }
     }
-    __syncthreads();
+    if (__syncthreads_or(nan_seen) && tid == 0) flag_status(ASP_DEV_NAN_SCORE);
     packed = s_overflow == 0;
     kcache = packed && 2 * n_packed <= pe - pb;
     if (!done && packed) {   // the candidates' second digit, from the packed lists

@@ -86,6 +86,9 @@ WORKLOADS: Dict[str, Workload] = {
         Workload("longcot_ragged_paged_b8", 8, 32, 8, 128, 65536, 8192, "bf16", 16, 2048, (4, 8, 16), 1e-2, 0.9, 3,
                  page_size=16,
                  description="the ragged paged workload with 8 sequences (a profiling-size case, ~1.2 GB of K/V)"),
+        Workload("qwen3_8b_shaped_b32_8k", 32, 32, 8, 128, 8192, 8192, "bf16", 16, 2048, (4, 8, 16), 1e-2, 0.9, 4,
+                 description="Qwen3-8B head geometry, batch 32, T=8192, C=2048 (a profiling-size case with the "
+                             "ragged batch's 200+ attention tiles per SM, ~1.1 GB of K/V)"),
         Workload("quest_page_scan_8b_32k", 8, 32, 8, 128, 32768, 32768, "bf16", 16, 2048, (4, 8, 16), 1e-2, 0.9, 1,
                  page_size=16,
                  description="Qwen3-8B shapes for the page-scan comparison path, 16-token pages"),

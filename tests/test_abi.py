@@ -58,7 +58,8 @@ def test_struct_layout_matches_the_c_compiler():
 int main(void) {
   printf("asp_kv %zu %zu %zu %zu %zu\n", sizeof(asp_kv), offsetof(asp_kv, k), offsetof(asp_kv, page_size),
          offsetof(asp_kv, page_table), offsetof(asp_kv, seq_lens));
-  printf("asp_pred_cfg %zu %zu %zu\n", sizeof(asp_pred_cfg), offsetof(asp_pred_cfg, windows), offsetof(asp_pred_cfg, lambda));
+  printf("asp_pred_cfg %zu %zu %zu %zu\n", sizeof(asp_pred_cfg), offsetof(asp_pred_cfg, windows), offsetof(asp_pred_cfg, lambda),
+         offsetof(asp_pred_cfg, pool));
   printf("asp_decode_args %zu %zu %zu %zu %zu %zu %zu\n", sizeof(asp_decode_args), offsetof(asp_decode_args, kv),
          offsetof(asp_decode_args, workspace_bytes), offsetof(asp_decode_args, s_main), offsetof(asp_decode_args, timing),
          offsetof(asp_decode_args, k_new), offsetof(asp_decode_args, quest_page));
@@ -75,13 +76,13 @@ int main(void) {
         lines = dict((ln.split()[0], [int(x) for x in ln.split()[1:]]) for ln in subprocess.check_output([exe], text=True).splitlines())
     K, P, D = L.AspKv, L.AspPredCfg, L.AspDecodeArgs
     assert lines["asp_kv"] == [ctypes.sizeof(K), K.k.offset, K.page_size.offset, K.page_table.offset, K.seq_lens.offset]
-    assert lines["asp_pred_cfg"] == [ctypes.sizeof(P), P.windows.offset, P.lam.offset]
+    assert lines["asp_pred_cfg"] == [ctypes.sizeof(P), P.windows.offset, P.lam.offset, P.pool.offset]
     assert lines["asp_decode_args"] == [ctypes.sizeof(D), D.kv.offset, D.workspace_bytes.offset, D.s_main.offset,
                                         D.timing.offset, D.k_new.offset, D.quest_page.offset]
 
 
 def test_version_and_status_strings(lib):
-    assert lib.asp_abi_version() == 2
+    assert lib.asp_abi_version() == 3
     assert L.status_string(L.ASP_OK) == "ok"
     assert "workspace" in L.status_string(L.ASP_ERR_WORKSPACE)
     assert L.status_string(99) == "unknown status"
@@ -226,9 +227,9 @@ def test_workspace_grows_with_the_tail(lib):
     assert b >= a
 
 
-def _cfg(W=16, windows=(4, 8, 16), lam=1e-2, coef=0):
+def _cfg(W=16, windows=(4, 8, 16), lam=1e-2, coef=0, pool=0):
     arr = (ctypes.c_int * len(windows))(*windows)
-    cfg = L.AspPredCfg(W, ctypes.cast(arr, ctypes.POINTER(ctypes.c_int)), len(windows), lam, coef)
+    cfg = L.AspPredCfg(W, ctypes.cast(arr, ctypes.POINTER(ctypes.c_int)), len(windows), lam, coef, pool)
     return cfg, arr
 
 
@@ -238,6 +239,7 @@ def _cfg(W=16, windows=(4, 8, 16), lam=1e-2, coef=0):
     (dict(lam=0.0), 0, L.ASP_ERR_INVALID_ARG),
     (dict(lam=-1.0), 0, L.ASP_ERR_INVALID_ARG),
     (dict(coef=3), 0, L.ASP_ERR_INVALID_ARG),
+    (dict(pool=2), 0, L.ASP_ERR_INVALID_ARG),
     (dict(W=40, windows=(4,)), 0, L.ASP_ERR_UNSUPPORTED),
     (dict(), 17, L.ASP_ERR_INVALID_ARG),
     (dict(), -1, L.ASP_ERR_INVALID_ARG),
@@ -260,6 +262,12 @@ def test_decode_step_and_wait_validation(lib):
     a = L.AspDecodeArgs()   # all zero: no query, no cache
     assert lib.asp_decode_step(ctypes.byref(a)) == L.ASP_ERR_INVALID_ARG
     assert lib.asp_wait_selection(None, 10) == L.ASP_ERR_INVALID_ARG
+
+
+def test_wait_limit_check_validation(lib):
+    assert lib.asp_check_wait_limit(8, None, None) == L.ASP_ERR_INVALID_ARG
+    assert lib.asp_check_wait_limit(0, FAKE, None) == L.ASP_ERR_INVALID_ARG
+    assert lib.asp_check_wait_limit((1 << 20) + 1, FAKE, None) == L.ASP_ERR_INVALID_ARG
 
 
 def test_quest_validation(lib):

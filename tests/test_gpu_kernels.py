@@ -74,16 +74,19 @@ def test_score_keys(dtype, d, G, page_size):
     qpred = torch.randn(B, Hkv * G, d, generator=_gen(5)).to(DEV)
     scores = torch.full((B, Hkv, T), float("nan"), device=DEV)
     asp.score_keys(qpred, kv, scores)
+    # the CUDA-core scan (the tensor-core scan's comparison for bf16 keys) gives the same scores
+    scores_cc = torch.full((B, Hkv, T), float("nan"), device=DEV)
+    asp.score_keys_cuda_cores(qpred, kv, scores_cc)
     torch.cuda.synchronize()
     keys, _ = host_sequences(kvd)
     ref = oracle.score_keys(np64(qpred), [keys[b] for b in range(B)], T)
-    got = scores.cpu().numpy()
-    for b in range(B):
-        for h in range(Hkv):
-            Tb = lens[b]
-            assert_scores_close(got[b, h, :Tb], ref[b, h, :Tb], np64(qpred[b, h * G:(h + 1) * G]), keys[b][h],
-                                what=f"b{b} h{h}")
-            assert np.isnan(got[b, h, Tb:]).all()      # entries past T_b are not written
+    for got in (scores.cpu().numpy(), scores_cc.cpu().numpy()):
+        for b in range(B):
+            for h in range(Hkv):
+                Tb = lens[b]
+                assert_scores_close(got[b, h, :Tb], ref[b, h, :Tb], np64(qpred[b, h * G:(h + 1) * G]),
+                                    keys[b][h], what=f"b{b} h{h}")
+                assert np.isnan(got[b, h, Tb:]).all()      # entries past T_b are not written
 
 
 _MANY_SHORT = [int(x) for x in np.random.default_rng(3).integers(1, 41, 200)]
@@ -388,7 +391,8 @@ def test_attend_flags_out_of_range_indices_and_skips_them():
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("W,windows", [(1, (1,)), (8, (4, 8)), (16, (4, 8, 16)), (16, (2, 5, 11)), (32, (1, 7, 32))])
 @pytest.mark.parametrize("coef", ["softmax", "raw"])
-def test_predict_query(d, W, windows, coef):
+@pytest.mark.parametrize("pool", ["predictions", "features"])
+def test_predict_query(d, W, windows, coef, pool):
     B, Hq = 2, 6
     g = _gen(W * 100 + d)
     q = [torch.randn(B, Hq, d, generator=g)]
@@ -400,10 +404,11 @@ def test_predict_query(d, W, windows, coef):
         slots = torch.roll(hist, shifts=ring, dims=2)      # slot (ring + s) % (W+1) holds s-th oldest
         qhist = slots.contiguous().to(DEV)
         qpred = torch.empty(B, Hq, d, device=DEV)
-        cfg = asp.PredCfg(W, windows, 1e-2, coef)
+        cfg = asp.PredCfg(W, windows, 1e-2, coef, pool)
         asp.predict_query(qhist, ring, cfg, qpred)
         torch.cuda.synchronize()
-        ref = oracle.predict_query(hist.double().numpy(), windows, 1e-2, coef)
+        fn = oracle.predict_query if pool == "predictions" else oracle.predict_query_pooled
+        ref = fn(hist.double().numpy(), windows, 1e-2, coef)
         assert_pred_close(qpred.cpu().numpy(), ref, f"W{W} {windows} ring{ring} {coef}")
         assert torch.equal(qhist.cpu(), slots)             # read-only without q_new
 
@@ -483,3 +488,39 @@ def test_wait_selection_times_out_then_completes():
         ev.record(s)
     assert asp.wait_selection(ev, 10) == asp._lib.ASP_ERR_TIMEOUT
     assert asp.wait_selection(ev, 30_000_000) == asp._lib.ASP_OK
+
+
+@pytest.mark.parametrize("T", [5000, 100003])
+def test_select_flags_nan_scores(T):
+    """NaN scores are invalid input: the selection reports them (ASP_DEV_NAN_SCORE)
+    and still writes a valid, bounded selection."""
+    C = 300
+    s = score_rows(2, T, seed=T)
+    s[1, 17] = float("nan")
+    s[1, T - 3] = float("nan")
+    sc = s.to(DEV).view(2, 1, T).contiguous()
+    idx = torch.full((2, 1, C), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.full((2, 1), -7, dtype=torch.int32, device=DEV)
+    assert asp.device_status() == 0
+    asp.select_topk(sc, None, C, idx, cnt)
+    bits = asp.device_status()
+    assert bits & asp.ASP_DEV_NAN_SCORE
+    got = idx.cpu().numpy()
+    assert cnt.cpu().tolist() == [[C], [C]]
+    for r in range(2):
+        assert np.all(np.diff(got[r, 0]) > 0) and got[r, 0].min() >= 0 and got[r, 0].max() < T
+    # the row without a NaN is still the exact top C
+    ref_idx, _ = oracle.select_topk(s[:1].numpy()[:, None, :], [T], C)
+    assert np.array_equal(got[0], ref_idx[0])
+
+
+def test_bounded_wait_gives_up_and_reports_it():
+    """The bounded barrier wait of every kernel, cut to a few attempts on a barrier
+    that nothing arrives on: the kernel gives up, records ASP_DEV_WAIT_LIMIT and
+    returns (no fault, no hang)."""
+    ret = torch.zeros(1, dtype=torch.int32, device=DEV)
+    assert asp.device_status() == 0
+    asp.check_wait_limit(64, ret)
+    torch.cuda.synchronize()
+    assert ret.item() == 1
+    assert asp.device_status() == asp.ASP_DEV_WAIT_LIMIT

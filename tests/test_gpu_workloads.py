@@ -347,3 +347,85 @@ def test_graph_replay_reproduces_eager_steps_bit_for_bit():
     assert states[1][1].ring_start == states[0][1].ring_start and states[1][1].cur == states[0][1].cur
     states[1][1].release_graphs()
     assert asp.device_status() == 0
+
+
+def test_dense_attention_bf16_at_the_8b_shape():
+    """Full attention (the pages' other baseline) as the bench times it: bf16, every
+    one of the 32768 cached tokens through the tail path (count 0, tail_begin 0),
+    sampled units against the oracle's dense softmax attention."""
+    wl = synth.workload("qwen3_8b_shaped_32k")
+    kvd = synth.kv_cache(wl, DEV)
+    B, Hq, Hkv, d, T = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.t_max
+    G = Hq // Hkv
+    kv = asp.KV(kvd["k"], kvd["v"], kvd["seq_lens"], t_max=T)
+    q = synth.query_history(wl, steps=1)[1][0].to(torch.bfloat16).to(DEV)
+    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty(B, Hq, device=DEV)
+    zero = torch.zeros(B, dtype=torch.int32, device=DEV)
+    ws = torch.empty(max(16, asp.attend_workspace_bytes(B, Hq, Hkv, d, 0, T)), dtype=torch.uint8, device=DEV)
+    asp.sparse_attend(q, kv, None, None, 0, out, lse, zero, T, ws)
+    torch.cuda.synchronize()
+    assert asp.device_status() == 0
+    units = [(0, 0), (3, 5), (7, 7)]
+    keys, vals = host_sequences(kvd, sorted({b for b, _ in units}))
+    qn = np64(q)
+    for b, h in units:
+        ref_o, ref_l = oracle.attend_set(qn[b, h * G:(h + 1) * G], keys[b][h], vals[b][h], np.arange(T))
+        assert_out_close(out[b, h * G:(h + 1) * G], ref_o, torch.bfloat16, f"dense b{b}h{h}")
+        assert_lse_close(lse[b, h * G:(h + 1) * G], ref_l)
+
+
+def test_layer_stack_gives_each_layer_its_single_step_results():
+    """Three layers decoded as the bench's stack does (every layer's attention on the
+    main stream in layer order, every layer's selection chain on one shared side
+    stream): each layer's output and next selection equal those of the same layer
+    stepped alone, bit for bit, and one layer matches the oracle."""
+    B, Hkv, G, d, T, C, W, windows = 2, 8, 4, 128, 4096, 256, 8, (4, 8)
+    Hq = Hkv * G
+    from test_gpu_kernels import make_cache
+
+    def layer(l):
+        kvd, kv = make_cache(B, Hkv, d, T, torch.bfloat16, [T, 3000], 0, seed=60 + l)
+        g = torch.Generator().manual_seed(70 + l)
+        qhist = torch.randn(B, Hq, W + 1, d, generator=g)
+        q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+        idx0, cnt0 = synth.random_selection(B, Hkv, C, [T, 3000], seed=80 + l)
+        return kvd, kv, qhist, q, idx0, cnt0
+
+    layers = [layer(l) for l in range(3)]
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream(priority=-100)
+    stacked, alone = [], []
+    for shared in (True, False):
+        for l, (kvd, kv, qhist, q, idx0, cnt0) in enumerate(layers):
+            st = asp.DecodeState(kv, Hq, asp.PredCfg(W, windows, 1e-2), C, qhist.to(DEV).contiguous(),
+                                 s_main=main, s_side=side if shared else None)
+            st.set_selection(idx0.to(DEV), cnt0.to(DEV))
+            out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=DEV)
+            (stacked if shared else alone).append((st, out))
+        states = stacked if shared else alone
+        for l, (st, out) in enumerate(states):   # one token through the stack (or each layer on its own)
+            st.step(layers[l][3].to(DEV), out)
+            if not shared:
+                main.wait_event(st.ev_sel_done)
+        for st, _ in states:
+            main.wait_event(st.ev_sel_done)
+        torch.cuda.synchronize()
+    assert asp.device_status() == 0
+    for (sa, oa), (sb, ob) in zip(stacked, alone):
+        assert torch.equal(oa, ob)
+        for x, y in zip(sa.selection, sb.selection):
+            assert torch.equal(x, y)
+    # layer 1 against the oracle's step
+    kvd, kv, qhist, q, idx0, cnt0 = layers[1]
+    keys, vals = host_sequences(kvd)
+    r = oracle.decode_step(q.double().numpy(), qhist.numpy(), [keys[0], keys[1]], [vals[0], vals[1]], idx0.numpy(),
+                           cnt0.numpy(), C, windows, 1e-2, T)
+    st, out = stacked[1]
+    assert_out_close(out, r["out"], torch.bfloat16, "stack layer 1")
+    assert_pred_close(st.qpred.cpu().numpy(), r["qpred"], "stack layer 1")
+    scores = st.scores.cpu().numpy()
+    idx1, cnt1 = (t.cpu().numpy() for t in st.selection)
+    for b, Tb in enumerate([T, 3000]):
+        for h in range(Hkv):
+            assert_valid_topk(scores[b, h], Tb, C, idx1[b, h], int(cnt1[b, h]), f"stack b{b}h{h}")
