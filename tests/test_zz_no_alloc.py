@@ -33,10 +33,11 @@ def _noalloc(q, kv, idx, cnt, C, out, lse):
                                              torch.cuda.current_stream().cuda_stream)
 
 
-def test_noalloc_matches_the_workspace_entry_point_on_two_calls():
+@pytest.mark.parametrize("B,Hq,Hkv,d,T,C", [(8, 32, 8, 128, 4096, 2048), (64, 32, 8, 128, 1100, 1024)],
+                         ids=["per_item_kernel", "gather_kernel"])
+def test_noalloc_matches_the_workspace_entry_point_on_two_calls(B, Hq, Hkv, d, T, C):
     from query_predicted_token_b200 import build
     build.build()
-    B, Hq, Hkv, d, T, C = 8, 32, 8, 128, 4096, 2048
     need = asp.attend_workspace_bytes(B, Hq, Hkv, d, C)
     assert 0 < need <= (2 << 20)          # the partials do use scratch, and fit the fixed array
     k, v = _cache(B, Hkv, T, d, seed=5)
@@ -57,4 +58,13 @@ def test_noalloc_matches_the_workspace_entry_point_on_two_calls():
         err = (out.float() - ref.float()).abs().max().item()
         assert err <= OUT_ATOL, f"call {call}: max abs difference {err}"
         assert torch.allclose(lse, ref_lse, rtol=1e-5, atol=1e-4), f"call {call}: lse"
+    # and one unit of the last call against the oracle's attention over the same rows
+    import oracle
+    G = Hq // Hkv
+    b, h = B - 1, Hkv - 1
+    K, V = k[b, h].double().cpu().numpy(), v[b, h].double().cpu().numpy()
+    S = idx[b, h, :int(cnt[b, h])].cpu().numpy()
+    ref_o, _ = oracle.attend_set(q[b, h * G:(h + 1) * G].double().cpu().numpy(), K, V, S)
+    err = (out[b, h * G:(h + 1) * G].double().cpu().numpy() - ref_o).__abs__().max()
+    assert err <= OUT_ATOL, f"against the oracle: {err}"
     assert asp.device_status() == 0
