@@ -481,6 +481,247 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectArgs a) {
   if (tid == 0) a.count[row] = out_stride - (s_last_sel ? (n * E - T) : 0);
 }
 
+
+// ---- rows of up to 32K scores with the first digit's histogram given ---------
+//
+// The decode step's rows at contexts up to 32K.  Warp 0 stages the row in shared
+// memory with bulk copies while the CTA finds the threshold digit from the given
+// histogram.  Then every lane classifies 32 consecutive scores (lane l of warp w:
+// units 1024 w + 32 l .. + 31, its eight 16-byte vectors read in an order rotated
+// by the lane, so that a warp's reads spread over all banks) against the float
+// edges of the threshold bin, in one pass: two 32-bit masks per lane, in index
+// order, of the units above the bin and of the candidates inside it.  The work is
+// bound by instruction issue (32K scores on one SM), so that pass is the only one
+// over every score; the candidates, a few percent of the row, are re-read from
+// shared memory for their later digits (one shared atomic each) and their final
+// class.  The output positions come from population counts, one scan over the
+// lanes and one over the warps, and the writes walk the masks' set bits.
+constexpr int kRegSpan = 1024;                             // units per warp
+constexpr int kRegMaxUnits = kWarps * kRegSpan;            // 32768
+constexpr uint32_t kRowPiece = 16384;                      // bytes per bulk copy
+
+// The float at or above which a score's key reaches k + 2^shift (the upper edge of
+// the bin of width 2^shift starting at k); NaN (no score) past the top key.
+__device__ __forceinline__ float edge_above(uint32_t k, int shift) {
+  const uint32_t e = k + (1u << shift);
+  return e < k ? __uint_as_float(0x7fc00000u) : key_edge(e);
+}
+
+// max that propagates NaN (one operand NaN gives NaN)
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// The digit (of width nb, bins taken two (or one) per thread, highest first) that
+// holds the krem-th largest counted key; on return krem is the count still needed
+// from that bin, and the result says whether the bin holds exactly that many.
+__device__ __forceinline__ bool regs_find_digit(const int (&v)[2], int nb, int shift, int& krem, uint32_t& prefix,
+                                                uint32_t& mask, int* wsum, int* s_res) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bpt = nb / kThreads;
+  const int local = v[0] + (bpt > 1 ? v[1] : 0);
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int wincl = wsum[lane];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, wincl, o);
+    if (lane >= o) wincl += y;
+  }
+  const int wbase = __shfl_sync(0xffffffffu, wincl - wsum[lane], warp);
+  const int excl = wbase + incl - local;
+  if (excl < krem && krem <= excl + local) {
+    const int j = (bpt > 1 && excl + v[0] < krem) ? 1 : 0;
+    s_res[0] = nb - 1 - (tid * bpt + j);   // the digit
+    s_res[1] = j ? excl + v[0] : excl;     // counted keys above its bin
+    s_res[2] = v[j];                       // keys in its bin
+  }
+  __syncthreads();
+  // s_res and wsum are written again only after the next search's first barrier
+  krem -= s_res[1];
+  prefix |= (uint32_t)s_res[0] << shift;
+  mask |= ((uint32_t)nb - 1u) << shift;
+  return s_res[2] == krem;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) select_regs_kernel(SelectArgs a) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int row = blockIdx.x;
+  const int b = row / a.rows_per_seq;
+  pdl_wait();   // the scores and their histogram come from the previous kernel
+
+  extern __shared__ __align__(16) float srow_s[];   // the row, rounded up to 4 scores
+  __shared__ int h1[kBins];    // second digit (11 bits)
+  __shared__ int h2[1024];     // third digit (10 bits)
+  __shared__ int wsum[kWarps];
+  __shared__ int wg[kWarps], we[kWarps];
+  __shared__ int s_res[3];
+  __shared__ uint64_t s_bar;
+
+  int T = a.seq_lens ? a.seq_lens[b] : a.t_max;
+  T = T < 0 ? 0 : (T > a.t_max ? a.t_max : T);
+  const int n = T;   // units are tokens (expand == 1)
+  const int C = a.c_units;
+  int32_t* out = a.idx + (size_t)row * C;
+  if (n <= C) {   // every token chosen
+    for (int u = tid; u < C; u += kThreads) out[u] = u < n ? u : -1;
+    if (tid == 0) a.count[row] = n;
+    return;
+  }
+
+  const float* srow = a.scores + (size_t)row * a.row_stride;
+  const uint32_t row_bytes = (uint32_t)((n + 3) & ~3) * 4u;   // inside the row: row_stride is a multiple of 4
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_init(&s_bar, 1);
+      mbar_init_fence();
+      mbar_arrive_expect_tx(&s_bar, row_bytes);
+    }
+    __syncwarp();
+    for (uint32_t off = (uint32_t)lane * kRowPiece; off < row_bytes; off += 32u * kRowPiece)
+      bulk_g2s(reinterpret_cast<uint8_t*>(srow_s) + off, reinterpret_cast<const uint8_t*>(srow) + off,
+               min(kRowPiece, row_bytes - off), &s_bar);
+  }
+  // bins 2047 - 2 tid and 2046 - 2 tid of the first digit: one 8-byte load
+  int hv[2];
+  {
+    const int* hp = a.hist0 + (size_t)row * kBins + (kBins - 2 - 2 * tid);
+    asm volatile("ld.global.v2.s32 {%0, %1}, [%2];" : "=r"(hv[1]), "=r"(hv[0]) : "l"(hp));
+  }
+  for (int i = tid; i < kBins; i += kThreads) h1[i] = 0;   // ordered by the digit search's barriers
+  for (int i = tid; i < 1024; i += kThreads) h2[i] = 0;
+  uint32_t prefix = 0u, mask = 0u;
+  int krem = C;
+  bool done = regs_find_digit(hv, kBins, kTopShift, krem, prefix, mask, wsum, s_res);
+  const float lo0 = key_edge(prefix), hi0 = edge_above(prefix, kTopShift);
+
+  const bool landed = mbar_wait(&s_bar, 0);
+  if (!__syncthreads_and(landed)) return;   // ASP_DEV_WAIT_LIMIT recorded
+
+  // ---- the one pass over the row: bit 4k + c of gk / ck is the unit of vector
+  // (k + lane) mod 8, element c; a rotation by 4 (lane mod 8) puts the bits in index
+  // order (bit j: unit base + j)
+  const int base = warp * kRegSpan + lane * 32;
+  uint32_t gmask = 0u, cmask = 0u;   // above the threshold bin / inside it
+  bool nan_seen = false;
+  if (base + 32 <= n) {
+    const float4* r4 = reinterpret_cast<const float4*>(srow_s + base);
+    float nacc = 0.f;
+    uint32_t gk = 0u, ck = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 x = r4[(k + lane) & 7];
+      const float xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        nacc = max_nan(nacc, xv[c]);
+        if (xv[c] >= hi0) gk |= 1u << (4 * k + c);
+        if (xv[c] >= lo0) ck |= 1u << (4 * k + c);
+      }
+    }
+    const int rot = 4 * (lane & 7);
+    gmask = __funnelshift_l(gk, gk, rot);
+    cmask = __funnelshift_l(ck, ck, rot) & ~gmask;
+    nan_seen = isnan(nacc);
+  } else if (base < n) {   // the lane that holds the end of the row
+    for (int j = 0; j < n - base; ++j) {
+      const float x = srow_s[base + j];
+      nan_seen |= isnan(x);
+      if (x >= hi0) gmask |= 1u << j;
+      else if (x >= lo0) cmask |= 1u << j;
+    }
+  }
+  // the candidates' later digits, from their scores in shared memory
+  auto key_of = [&](int j) -> uint32_t { return order_key(srow_s[base + j]); };
+  if (!done) {
+    for (uint32_t m = cmask; m; m &= m - 1u) atomicAdd(&h1[(key_of(__ffs(m) - 1) >> 10) & 2047u], 1);
+  }
+  if (__syncthreads_or(nan_seen) && tid == 0) flag_status(ASP_DEV_NAN_SCORE);
+  if (!done) {
+    const int hb[2] = {h1[kBins - 1 - 2 * tid], h1[kBins - 2 - 2 * tid]};
+    done = regs_find_digit(hb, kBins, 10, krem, prefix, mask, wsum, s_res);
+    if (!done) {   // the third digit (10 bits): the rest of the key
+      const uint32_t p1 = prefix, m1 = mask;
+      for (uint32_t m = cmask; m; m &= m - 1u) {
+        const uint32_t key = key_of(__ffs(m) - 1);
+        if ((key & m1) == p1) atomicAdd(&h2[key & 1023u], 1);
+      }
+      __syncthreads();
+      const int hb2[2] = {h2[1023 - tid], 0};
+      regs_find_digit(hb2, 1024, 0, krem, prefix, mask, wsum, s_res);
+    }
+  }
+
+  // ---- output: the units above the threshold, and the first krem of those at it
+  // (all of them when the bin holds exactly krem), lowest index first, ascending
+  uint32_t emask = cmask;   // at the threshold
+  if (mask != (((uint32_t)kBins - 1u) << kTopShift)) {   // later digits: sort the candidates
+    emask = 0u;
+    for (uint32_t m = cmask; m; m &= m - 1u) {
+      const int j = __ffs(m) - 1;
+      const uint32_t mk = key_of(j) & mask;
+      if (mk > prefix) gmask |= 1u << j;
+      else if (mk == prefix) emask |= 1u << j;
+    }
+  }
+  const int cg = __popc(gmask), ce = __popc(emask);
+  int ig = cg, ie = ce;   // inclusive scans over the lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int yg = __shfl_up_sync(0xffffffffu, ig, o);
+    const int ye = __shfl_up_sync(0xffffffffu, ie, o);
+    if (lane >= o) {
+      ig += yg;
+      ie += ye;
+    }
+  }
+  if (lane == 31) {
+    wg[warp] = ig;
+    we[warp] = ie;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int g = wg[lane], e = we[lane];
+    int gi = g, ei = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yg = __shfl_up_sync(0xffffffffu, gi, o);
+      const int ye = __shfl_up_sync(0xffffffffu, ei, o);
+      if (lane >= o) {
+        gi += yg;
+        ei += ye;
+      }
+    }
+    wg[lane] = gi - g;   // exclusive offsets of the warps
+    we[lane] = ei - e;
+  }
+  __syncthreads();
+  int G = wg[warp] + ig - cg, E = we[warp] + ie - ce;   // units of each kind before this lane's
+  uint32_t m = gmask | (E < krem ? emask : 0u);
+  while (m) {
+    const int j = __ffs(m) - 1;
+    m &= m - 1u;
+    const bool g = (gmask >> j) & 1u;
+    const int pos = G + min(E, krem);
+    if (pos < C) {
+      out[pos] = base + j;
+    } else {   // only reachable with a histogram that does not match the scores
+      flag_status(ASP_DEV_SELECT);
+    }
+    if (g) ++G; else ++E;
+    if (E >= krem) m &= gmask;   // the quota of ties is filled
+  }
+  if (tid == 0) a.count[row] = C;
+}
+
 }  // namespace
 
 bool select_supported(int t_max, int expand) { return t_max >= 1 && expand >= 1; }
@@ -493,6 +734,11 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)(args.key_cap > 0 ? args.key_cap : 4) * 4;
   const bool fused = a.hist0 != nullptr && (a.row_stride & 3) == 0 &&
                      (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0 && args.key_cap >= kWarps * 4;
+  if (fused && a.expand == 1 && a.t_max <= kRegMaxUnits) {
+    const size_t row_smem = (size_t)((a.t_max + 3) & ~3) * 4;
+    if (prepare_kernel((const void*)select_regs_kernel, row_smem, kThreads) < 1) return cudaErrorInvalidConfiguration;
+    return launch_pdl(select_regs_kernel, dim3(args.n_rows), dim3(kThreads), row_smem, s, args);
+  }
   auto kern = fused ? select_kernel<true> : select_kernel<false>;
   if (prepare_kernel((const void*)kern, smem, kThreads) < 1) return cudaErrorInvalidConfiguration;
   return launch_pdl(kern, dim3(args.n_rows), dim3(kThreads), smem, s, args);

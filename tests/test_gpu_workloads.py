@@ -228,6 +228,59 @@ def test_decode_selection_ties_across_the_halves_of_a_row():
     assert np.array_equal(idx, ref_idx)
 
 
+def test_decode_selection_up_to_32k_tokens_matches_the_oracle_on_ragged_rows():
+    """Rows of at most 32K tokens keep the whole row in registers (one 16-byte vector
+    per lane and chunk): ragged lengths that end inside a vector, inside a warp's
+    span and exactly at C, and a row shorter than C, against the oracle's selection
+    over the same scores, index for index."""
+    B, Hkv, G, d, T, C = 5, 2, 2, 128, 32768, 2048
+    lens = torch.tensor([1000, 2048, 3001, 17003, 32768], dtype=torch.int32)
+    g = torch.Generator().manual_seed(21)
+    k = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).to(DEV)
+    v = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).to(DEV)
+    scores, idx, cnt = _decode_once(k, v, lens, Hkv * G, C)
+    ref_idx, ref_cnt = oracle.select_topk(scores, lens.tolist(), C)
+    assert np.array_equal(cnt, ref_cnt)
+    assert np.array_equal(idx, ref_idx)
+
+
+def test_decode_selection_up_to_32k_tokens_of_tied_scores():
+    """Every score equal on rows of at most 32K tokens: the first C tokens of each row
+    (the first digit's bin holds the whole row, and the third digit still leaves
+    exact ties, taken lowest index first)."""
+    B, Hkv, G, d, T, C = 4, 2, 2, 128, 32768, 2048
+    lens = torch.tensor([1000, 2048, 20001, 32768], dtype=torch.int32)
+    k = torch.zeros(B, Hkv, T, d, dtype=torch.bfloat16, device=DEV)
+    v = torch.zeros(B, Hkv, T, d, dtype=torch.bfloat16, device=DEV)
+    scores, idx, cnt = _decode_once(k, v, lens, Hkv * G, C)
+    for b in range(B):
+        n = min(C, int(lens[b]))
+        for h in range(Hkv):
+            assert int(cnt[b, h]) == n
+            assert idx[b, h, :n].tolist() == list(range(n)), f"b{b}h{h}"
+            assert np.all(idx[b, h, n:] == -1)
+
+
+def test_decode_selection_up_to_32k_tokens_with_few_distinct_scores():
+    """Keys drawn from eight vectors give eight score values per row, so the C-th
+    largest sits inside a group of exactly equal scores that the three digits cannot
+    split: the group's first tokens by index fill the quota, as in the oracle."""
+    B, Hkv, G, d, T, C = 2, 2, 2, 128, 30000, 5000
+    lens = torch.tensor([30000, 24001], dtype=torch.int32)
+    g = torch.Generator().manual_seed(23)
+    basis = torch.randn(8, d, generator=g)
+    pick = torch.randint(0, 8, (B, Hkv, T), generator=g)
+    k = basis[pick].to(torch.bfloat16).to(DEV)
+    v = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).to(DEV)
+    scores, idx, cnt = _decode_once(k, v, lens, Hkv * G, C)
+    for b in range(B):
+        for h in range(Hkv):
+            assert np.unique(scores[b, h, :lens[b]]).size <= 8
+    ref_idx, ref_cnt = oracle.select_topk(scores, lens.tolist(), C)
+    assert np.array_equal(cnt, ref_cnt)
+    assert np.array_equal(idx, ref_idx)
+
+
 def test_decode_selection_when_most_tokens_survive_the_first_digit():
     """C close to T_b on rows longer than the selection's shared memory: the survivors
     of the first digit overflow the packed lists and the row is re-read from L2."""
