@@ -48,7 +48,7 @@
 extern "C" {
 #endif
 
-#define ASP_ABI_VERSION 3
+#define ASP_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define ASP_API __attribute__((visibility("default")))
@@ -234,6 +234,11 @@ ASP_API size_t asp_attend_workspace_bytes(int batch, int n_q_heads, int n_kv_hea
 ASP_API size_t asp_decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C,
                                           int max_tail);
 
+/* Bytes of one predictor-factor buffer of asp_decode_step (pred_factor_cur / _next):
+ * per query head the scaled rows of the lag Gram's Cholesky factor and its inverse
+ * diagonal, fp64.  0 for invalid arguments. */
+ASP_API size_t asp_pred_factor_bytes(int batch, int n_q_heads, const asp_pred_cfg* cfg);
+
 /* ---------------------------------------------------------------------------
  * Step 4 without a caller-provided workspace.  No counterpart in the paper: this
  * entry point exists for callers that cannot allocate device memory -- for example
@@ -331,6 +336,24 @@ typedef struct {
   const void* v_new;
   void* quest_meta;             /* NULL, or page bounds kept current (see asp_append_kv) */
   int quest_page;
+  /* Optional: the predictor's lag factorisation moved off the critical path.  The
+   * lag Gram that step t+1 solves holds q_t and the W - 1 queries before it, all
+   * known at step t, so step t factorises it into pred_factor_next on s_main once
+   * its key scan is done (ev_fork is then recorded again on s_side after the scan),
+   * beside the selection, and step t+1's predictor only forms the right-hand side
+   * and substitutes.  Both buffers hold asp_pred_factor_bytes(...) bytes (8-byte
+   * aligned, distinct); the caller swaps them between steps like idx_cur/idx_next
+   * and sets pred_factor_valid = 1 once pred_factor_cur holds the factor the
+   * previous decode step wrote for this ring (0 on a first step or after the ring
+   * was changed otherwise: the step then factorises in full).  NULL pointers turn
+   * the precomputation off.  It is also off (every step factorises in full, the
+   * buffers untouched) when the selection's CTAs (batch * n_kv_heads) and the
+   * factorisation's (one per 4 query heads) do not fit on the GPU's SMs together,
+   * for windows that are not powers of two filling at most 32 lags, and for the
+   * pooled-features reading. */
+  double* pred_factor_cur;
+  int pred_factor_valid;
+  double* pred_factor_next;
 } asp_decode_args;
 
 ASP_API asp_status asp_decode_step(const asp_decode_args* args);

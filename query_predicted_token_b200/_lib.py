@@ -43,7 +43,8 @@ class AspDecodeArgs(ctypes.Structure):
                 ("out", c_void_p), ("lse", c_void_p), ("workspace", c_void_p), ("workspace_bytes", c_size_t),
                 ("s_main", c_void_p), ("s_side", c_void_p), ("ev_fork", c_void_p), ("ev_sel_done", c_void_p),
                 ("timing", POINTER(c_void_p)), ("k_new", c_void_p), ("v_new", c_void_p), ("quest_meta", c_void_p),
-                ("quest_page", c_int)]
+                ("quest_page", c_int), ("pred_factor_cur", c_void_p), ("pred_factor_valid", c_int),
+                ("pred_factor_next", c_void_p)]
 
 
 SIGNATURES = {
@@ -55,6 +56,7 @@ SIGNATURES = {
                                   c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "asp_attend_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int]),
     "asp_decode_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int]),
+    "asp_pred_factor_bytes": (c_size_t, [c_int, c_int, POINTER(AspPredCfg)]),
     "asp_sparse_attend_noalloc": (c_int, [c_void_p, c_int, c_int, POINTER(AspKv), c_void_p, c_void_p, c_int, c_void_p,
                                           c_int, c_void_p, c_void_p, c_void_p]),
     "asp_decode_step": (c_int, [POINTER(AspDecodeArgs)]),
@@ -292,10 +294,15 @@ def event_handle(ev) -> int:
 class DecodeState:
     """Buffers of the asynchronous decode loop: the query ring, double-buffered
     selections, scratch for the side stream, attention workspace, two streams and
-    two events.  :meth:`step` is one ``asp_decode_step`` call."""
+    two events.  :meth:`step` is one ``asp_decode_step`` call.  With
+    ``precompute_factor`` each step also factorises the next step's lag Gram beside
+    its key scan (two double-buffered factor buffers), so that the next step's
+    predictor only substitutes; after changing ``qhist`` or ``ring_start`` outside
+    :meth:`step`, call :meth:`invalidate_factor`."""
 
     def __init__(self, kv: KV, n_q_heads: int, cfg: PredCfg, C: int, qhist: torch.Tensor, max_tail: int = 0,
-                 tail_begin: Optional[torch.Tensor] = None, s_main=None, s_side=None, timing: bool = False):
+                 tail_begin: Optional[torch.Tensor] = None, s_main=None, s_side=None, timing: bool = False,
+                 precompute_factor: bool = True):
         dev = kv.k.device
         B, Hkv, d = kv.batch, kv.n_kv_heads, kv.head_dim
         self.kv, self.cfg, self.C, self.n_q_heads = kv, cfg, int(C), int(n_q_heads)
@@ -309,6 +316,9 @@ class DecodeState:
         self.cur = 0
         ws = int(lib().asp_decode_workspace_bytes(B, n_q_heads, Hkv, d, C, max_tail if tail_begin is not None else 0))
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+        fb = int(lib().asp_pred_factor_bytes(B, n_q_heads, ctypes.byref(cfg.struct))) if precompute_factor else 0
+        self.pred_factor = [torch.empty(fb // 8, dtype=torch.float64, device=dev) for _ in range(2)] if fb else None
+        self._factor_valid = False
         self.s_main = s_main or torch.cuda.current_stream()
         # the selection chain is the step's critical path: give it the highest priority
         self.s_side = s_side or torch.cuda.Stream(priority=-100)
@@ -344,7 +354,14 @@ class DecodeState:
         a.ev_fork = event_handle(self.ev_fork)
         a.ev_sel_done = event_handle(self.ev_sel_done)
         a.timing = ctypes.cast(self._timing_arr, POINTER(c_void_p)) if self._timing_arr is not None else None
+        if self.pred_factor is not None:
+            a.pred_factor_cur = _ptr(self.pred_factor[cur])
+            a.pred_factor_next = _ptr(self.pred_factor[nxt])
         return a
+
+    def invalidate_factor(self) -> None:
+        """The next step factorises in full (the stored factor no longer matches the ring)."""
+        self._factor_valid = False
 
     def set_timing(self, on: bool) -> None:
         """Record the per-kernel timing events in later steps (they sit between the
@@ -374,7 +391,9 @@ class DecodeState:
         a.v_new = _ptr(v_new)
         a.quest_meta = _ptr(quest_meta)
         a.quest_page = int(quest_page)
+        a.pred_factor_valid = 1 if self._factor_valid else 0
         _check("asp_decode_step", self._fn(ctypes.byref(a)))
+        self._factor_valid = self.pred_factor is not None
         self.cur = 1 - self.cur
         self.ring_start = (self.ring_start + 1) % (self.cfg.W + 1)
 
@@ -389,7 +408,7 @@ class DecodeState:
         (the library prepares its kernels on first use).  Returns the cycle length."""
         import math
         n = 2 * (self.cfg.W + 1) // math.gcd(2, self.cfg.W + 1)
-        cur0, ring0 = self.cur, self.ring_start
+        cur0, ring0, fv0 = self.cur, self.ring_start, self._factor_valid
         main0 = self.s_main
         timing_on = bool(self._args[0].timing)
         cap = torch.cuda.Stream(device=self.kv.k.device)
@@ -412,7 +431,7 @@ class DecodeState:
             self.s_main = main0
             self._args = [self._build_args(0), self._build_args(1)]
             self.set_timing(timing_on) if self._timing_arr is not None else None
-            self.cur, self.ring_start = cur0, ring0
+            self.cur, self.ring_start, self._factor_valid = cur0, ring0, fv0
         # the events were last recorded inside the captures: record them once outside
         self.ev_fork.record(self.s_main)
         self.ev_sel_done.record(self.s_main)
@@ -430,6 +449,7 @@ class DecodeState:
         _check("asp_graph_launch", lib().asp_graph_launch(self.graphs[self._graph_at][1],
                                                           _stream(torch.cuda.current_stream())))
         self._graph_at = (self._graph_at + 1) % len(self.graphs)
+        self._factor_valid = self.pred_factor is not None
         self.cur = 1 - self.cur
         self.ring_start = (self.ring_start + 1) % (self.cfg.W + 1)
 

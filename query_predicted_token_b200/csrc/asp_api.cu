@@ -156,6 +156,9 @@ asp::PredictArgs predict_args(float* qhist, int ring_start, const void* q_new, a
   a.coef_raw = cfg->coef == ASP_COEF_RAW;
   a.pool_features = cfg->pool == ASP_POOL_FEATURES;
   a.qpred = qpred;
+  a.mode = 0;
+  a.factor_in = nullptr;
+  a.factor_out = nullptr;
   return a;
 }
 
@@ -273,6 +276,13 @@ size_t asp_decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int 
          (size_t)batch * n_kv_heads * asp::kTopBins * 4;
 }
 
+size_t asp_pred_factor_bytes(int batch, int n_q_heads, const asp_pred_cfg* cfg) {
+  if (batch <= 0 || n_q_heads <= 0 || check_pred(cfg, 0) != ASP_OK) return 0;
+  int wmax = 0;
+  for (int i = 0; i < cfg->n_windows; ++i) wmax = cfg->windows[i] > wmax ? cfg->windows[i] : wmax;
+  return asp::predict_factor_bytes(batch * n_q_heads, wmax);
+}
+
 size_t asp_attend_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int head_dim, int C, int max_tail) {
   if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || C < 0 || max_tail < 0 || (long)C + max_tail < 1) return 0;
   if (head_dim != 64 && head_dim != 128) return 0;
@@ -325,6 +335,10 @@ asp_status asp_decode_step(const asp_decode_args* a) {
   st = check_pred(a->pred, a->ring_start);
   if (st != ASP_OK) return st;
   if (!asp::select_supported(a->kv->t_max, 1) || a->kv->batch > kMaxScoreBatch) return ASP_ERR_UNSUPPORTED;
+  if ((a->pred_factor_cur && (reinterpret_cast<uintptr_t>(a->pred_factor_cur) & 7)) ||
+      (a->pred_factor_next && (reinterpret_cast<uintptr_t>(a->pred_factor_next) & 7)) ||
+      (a->pred_factor_cur && a->pred_factor_cur == a->pred_factor_next))
+    return ASP_ERR_INVALID_ARG;
   if (a->k_new) {   // the step appends the new token first: it writes seq_lens and tail_begin
     st = check_append(a->kv, a->k_new, a->v_new, a->quest_meta, a->quest_page);
     if (st != ASP_OK) return st;
@@ -333,6 +347,18 @@ asp_status asp_decode_step(const asp_decode_args* a) {
 
   cudaStream_t sm = reinterpret_cast<cudaStream_t>(a->s_main);
   cudaStream_t ss = reinterpret_cast<cudaStream_t>(a->s_side);
+  // The lag factorisation moves to the previous step when it can run beside the
+  // selection without taking SMs from it: the selection's CTAs (one per row) and
+  // the factorisation's (four heads each) fit on the GPU at once.  A pure function
+  // of the sizes, so consecutive steps agree on it.
+  bool use_factor = false;
+  {
+    asp::PredictArgs probe = predict_args(a->qhist, a->ring_start, a->q_t, a->q_dtype, a->kv->batch, a->n_q_heads,
+                                          a->kv->head_dim, a->pred, a->qpred);
+    const long rows = (long)a->kv->batch * a->kv->n_kv_heads;
+    const long fctas = ((long)a->kv->batch * a->n_q_heads + 3) / 4;
+    use_factor = asp::predict_factor_eligible(probe) && rows + fctas <= asp::sm_count();
+  }
   cudaEvent_t fork = reinterpret_cast<cudaEvent_t>(a->ev_fork);
   cudaEvent_t done = reinterpret_cast<cudaEvent_t>(a->ev_sel_done);
   auto mark = [&](int i, cudaStream_t s) -> cudaError_t {
@@ -366,6 +392,10 @@ asp_status asp_decode_step(const asp_decode_args* a) {
                                        a->kv->head_dim, a->pred, a->qpred);
     pa.zero = hist;   // the score kernel accumulates the selection's first histogram here
     pa.zero_words = hist_words;
+    if (use_factor && a->pred_factor_cur && a->pred_factor_valid) {
+      pa.mode = 2;
+      pa.factor_in = a->pred_factor_cur;
+    }
     e = asp::launch_predict(pa, ss);
   }
   if (e == cudaSuccess) e = mark(1, ss);
@@ -373,6 +403,18 @@ asp_status asp_decode_step(const asp_decode_args* a) {
   // the predictor is the scan's only producer in this stream: the scan may start
   // streaming keys while it runs
   if (e == cudaSuccess) e = asp::launch_score(a->qpred, a->n_q_heads, kv, a->scores, ss, hist, true);
+  // main stream, once the scan is done: the next step's lag factorisation, on the SMs
+  // the selection leaves free (it reads q_t and ring slots this step's push leaves
+  // alone); ev_fork is reused to carry the scan's completion
+  if (e == cudaSuccess && use_factor && a->pred_factor_next) {
+    e = cudaEventRecord(fork, ss);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sm, fork, 0);
+    asp::PredictArgs fa = predict_args(a->qhist, a->ring_start, a->q_t, a->q_dtype, B, a->n_q_heads,
+                                       a->kv->head_dim, a->pred, a->qpred);
+    fa.mode = 1;
+    fa.factor_out = a->pred_factor_next;
+    if (e == cudaSuccess) e = asp::launch_predict(fa, sm);
+  }
   if (e == cudaSuccess) e = mark(3, ss);
   if (e == cudaSuccess) e = mark(4, ss);
   if (e == cudaSuccess) {

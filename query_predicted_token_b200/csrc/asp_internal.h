@@ -89,8 +89,18 @@ struct PredictArgs {
   int pool_features;      // 1: regress on the windows' pooled features (the recorded alternative reading)
   float* qpred;
   int win_fast;           // set by launch_predict: windows sorted, powers of two, one round of lanes
+  // decode loop: 0 factorise and predict; 1 only factorise the next step's lag Gram
+  // into factor_out; 2 predict with factor_in (stored by the previous step's mode 1)
+  int mode;
+  const double* factor_in;
+  double* factor_out;
 };
 cudaError_t launch_predict(const PredictArgs& a, cudaStream_t s);
+// Whether the factor modes apply to these windows (powers of two in one round of
+// lanes, not the pooled-features reading); otherwise mode 2 predicts in full and
+// mode 1 launches nothing.
+bool predict_factor_eligible(const PredictArgs& a);
+size_t predict_factor_bytes(int n_heads, int wmax);
 
 // ---- step 2 -----------------------------------------------------------------
 struct KvView {

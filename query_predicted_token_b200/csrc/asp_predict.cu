@@ -98,14 +98,27 @@ struct GramRows {
 // FAST: the windows are powers of two that fit one warp (PredictArgs::win_fast);
 // the kernel for that case carries no code for the general one.  EXACT: the
 // widest window has NV - 1 lags, so every bound on the lags is a constant.
-template <int D, int NV, bool FAST, bool EXACT>
+// MODE (decode loop, FAST and EXACT only): the lag Gram of the next step holds
+// only queries that are known one step ahead -- the next step's lags are this
+// step's query and the W - 1 before it -- so its factorisation can run beside the
+// current step instead of on the next step's critical path.
+//   kPredFull:    factorise and predict (every other use);
+//   kPredFactor:  only factorise the next step's lag Gram (the current query
+//                 q_new becomes the newest lag) and store the factor;
+//   kPredUsing:   predict with the factor the previous step stored: only the
+//                 right-hand side (the lags' dot products with q_t) and the
+//                 substitutions remain.
+constexpr int kPredFull = 0, kPredFactor = 1, kPredUsing = 2;
+
+template <int D, int NV, bool FAST, bool EXACT, int MODE = kPredFull>
 __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(PredictArgs a) {
   constexpr int CPL = D / 32;   // contiguous channels per lane
   extern __shared__ __align__(16) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head = blockIdx.x * kWarps + warp;
+  static_assert(MODE == kPredFull || (FAST && EXACT), "the factor modes serve the decode loop's windows");
   pdl_trigger();   // the key scan may launch and run its prologue meanwhile
-  if (a.zero) {   // clear the next kernel's histogram (16-byte stores, spread over all warps)
+  if (MODE != kPredFactor && a.zero) {   // clear the next kernel's histogram (16-byte stores, spread over all warps)
     const size_t n4 = a.zero_words / 4;
     int4* z4 = reinterpret_cast<int4*>(a.zero);
     for (size_t i = (size_t)head * 32 + lane; i < n4; i += (size_t)gridDim.x * kWarps * 32) z4[i] = make_int4(0, 0, 0, 0);
@@ -129,7 +142,26 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
   for (int v = 0; v < NV; ++v) {
 #pragma unroll
     for (int c = 0; c < CPL; ++c) h[v][c] = 0.f;
-    if (v < n) {
+    if (MODE == kPredFactor) {
+      // the next step's vectors: h[0] (its target) unknown, h[1] = q_new, h[v >= 2] =
+      // q_{t+1-v}, in slot ring_start + 1 - v (not the slot the current step's push
+      // overwrites, so the two kernels may run at the same time)
+      if (v >= 1 && v < n) {
+        if (v == 1) {
+          const size_t off = (size_t)head * D + lane * CPL;
+#pragma unroll
+          for (int c = 0; c < CPL; ++c)
+            h[1][c] = a.q_new_f32 ? static_cast<const float*>(a.q_new)[off + c]
+                                  : __bfloat162float(static_cast<const __nv_bfloat16*>(a.q_new)[off + c]);
+        } else {
+          int slot = a.ring_start + 1 - v;
+          if (slot < 0) slot += nslot;
+          const float* src = hist + (size_t)slot * D + lane * CPL;
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) h[v][c] = src[c];
+        }
+      }
+    } else if (v < n) {
       // start <= nslot and 0 <= W - v <= W < nslot: one subtraction wraps the slot
       int slot = start + a.W - v;
       if (slot >= nslot) slot -= nslot;
@@ -149,22 +181,62 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
       }
     }
   }
-  if (a.q_new) {   // push q_t into the ring: it replaces the oldest slot (ring_start)
+  if (MODE != kPredFactor && a.q_new) {   // push q_t into the ring: it replaces the oldest slot (ring_start)
     float* dst = hist + (size_t)a.ring_start * D + lane * CPL;
 #pragma unroll
     for (int c = 0; c < CPL; ++c) dst[c] = h[0][c];
   }
 
-  // Gram of the n vectors: pairs (i, j), j <= i < NV, enumerated row by row, 32
-  // per round; after the reduce-scatter lane l holds pair (round base + l).
-  {
-    float part[32];
-    GramRows<NV, CPL, 0>::run(h, part, lane, wmax, a.lam, A, rhs);
-  }
-  __syncwarp();
-
   constexpr int WMAX = NV - 1;   // lags the registers can hold
   const int wm = wmax;
+  // the stored factor of one head: rows of L scaled by 1 / L_ii ([WMAX][WMAX], j < i),
+  // then the 1 / L_ii ([WMAX])
+  constexpr int kFac = WMAX * WMAX + WMAX;
+  if constexpr (MODE == kPredUsing) {
+    // right-hand side only: the lags' dot products with the target, reduced over
+    // the warp (lane r then holds rhs_r)
+    float part[32];
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      float acc = 0.f;
+      if (r < WMAX) {
+        acc = h[1 + r][0] * h[0][0];
+#pragma unroll
+        for (int c = 1; c < CPL; ++c) acc = fmaf(h[1 + r][c], h[0][c], acc);
+      }
+      part[r] = acc;
+    }
+    ReduceScatter<32, 16>::run(part, lane);
+    // forward substitution L z = rhs with the stored factor: z_i = rhs_i / L_ii -
+    // sum_{j<i} (L_ij / L_ii) z_j, one shuffle and one multiply-add per step
+    const double* fac = a.factor_in + (size_t)head * kFac;
+    double srow[WMAX];
+#pragma unroll
+    for (int j = 0; j < WMAX; ++j) srow[j] = (lane < WMAX && j < lane) ? fac[lane * WMAX + j] : 0.0;
+    const double my_inv = lane < WMAX ? fac[WMAX * WMAX + lane] : 0.0;
+    double zacc = lane < WMAX ? (double)part[0] * my_inv : 0.0;
+#pragma unroll
+    for (int k = 0; k < WMAX; ++k) {
+      const double zk = __shfl_sync(0xffffffffu, zacc, k);
+      if (lane > k) zacc = fma(-srow[k], zk, zacc);
+    }
+    // the factor goes where the back substitutions read it
+    if (lane < WMAX) {
+      invd[lane] = my_inv;
+#pragma unroll
+      for (int j = 0; j < WMAX; ++j)
+        if (j < lane) A[lane * kLda + j] = srow[j];
+    }
+    rhs[lane] = zacc;
+    __syncwarp();
+  } else {
+    // Gram of the n vectors: pairs (i, j), j <= i < NV, enumerated row by row, 32
+    // per round; after the reduce-scatter lane l holds pair (round base + l).
+    float part[32];
+    GramRows<NV, CPL, 0>::run(h, part, lane, wmax, a.lam, A, rhs);
+    __syncwarp();
+  }
+
   // Cholesky A = L L^T fused with the forward substitution L z = rhs.  Lane i
   // holds row i of A (then of L) and rhs_i (then z_i) in registers.  The chain
   // that bounds the loop is pivot -> 1/L_kk -> the next pivot: lane k+1 forms its
@@ -173,7 +245,7 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
   // shared memory, one store per lane and one broadcast load per later column).
   double z = lane < wm ? rhs[lane] : 0.0;
   double* col = invd + 32;
-  {
+  if constexpr (MODE != kPredUsing) {
     double arow[WMAX];
 #pragma unroll
     for (int j = 0; j < WMAX; ++j) arow[j] = (j <= lane && lane < wm && j < wm) ? A[lane * kLda + j] : 0.0;
@@ -213,6 +285,16 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
 #pragma unroll
       for (int j = 0; j < WMAX; ++j)
         if (j < lane) A[lane * kLda + j] = arow[j] * my_inv;
+    }
+    if constexpr (MODE == kPredFactor) {
+      double* fac = a.factor_out + (size_t)head * kFac;
+      if (lane < WMAX) {
+#pragma unroll
+        for (int j = 0; j < WMAX; ++j)
+          if (j < lane) fac[lane * WMAX + j] = arow[j] * my_inv;
+        fac[WMAX * WMAX + lane] = my_inv;
+      }
+      return;
     }
   }
   __syncwarp();
@@ -519,6 +601,12 @@ cudaError_t launch_t(const PredictArgs& a, cudaStream_t s) {
   const int grid = (a.n_heads + kWarps - 1) / kWarps;
   const size_t smem = kWarps * Solve<NV>::kBytes;
   const bool exact = a.wmax == NV - 1;
+  if (a.mode != kPredFull) {   // the decode loop's factor modes (see predict_factor_eligible)
+    auto kern = a.mode == kPredFactor ? predict_kernel<D, NV, true, true, kPredFactor>
+                                      : predict_kernel<D, NV, true, true, kPredUsing>;
+    if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
+    return launch_prio(kern, dim3(grid), dim3(kWarps * 32), smem, s, a);
+  }
   auto kern = a.win_fast ? (exact ? predict_kernel<D, NV, true, true> : predict_kernel<D, NV, true, false>)
                          : (exact ? predict_kernel<D, NV, false, true> : predict_kernel<D, NV, false, false>);
   if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
@@ -534,11 +622,9 @@ cudaError_t launch_d(const PredictArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_predict(const PredictArgs& args, cudaStream_t s) {
-  // The mean over the windows does not depend on their order: sort them widest
-  // first, so that windows whose widths are powers of two and add up to at most
-  // 32 lanes each start at a multiple of their width.
-  PredictArgs a = args;
+// Windows sorted widest first; whether they are powers of two filling at most one
+// round of lanes.
+static void sort_windows(PredictArgs& a) {
   for (int i = 1; i < a.n_win; ++i)
     for (int j = i; j > 0 && a.windows[j] > a.windows[j - 1]; --j) {
       const int t = a.windows[j];
@@ -552,6 +638,30 @@ cudaError_t launch_predict(const PredictArgs& args, cudaStream_t s) {
     pow2 = pow2 && a.windows[i] > 0 && (a.windows[i] & (a.windows[i] - 1)) == 0;
   }
   a.win_fast = (pow2 && sum <= 32) ? 1 : 0;
+}
+
+bool predict_factor_eligible(const PredictArgs& args) {
+  PredictArgs a = args;
+  sort_windows(a);
+  const int nv = a.wmax + 1 <= 9 ? 9 : (a.wmax + 1 <= 17 ? 17 : 33);
+  return !a.pool_features && a.win_fast && a.wmax == nv - 1;
+}
+
+size_t predict_factor_bytes(int n_heads, int wmax) {
+  const int nv = wmax + 1 <= 9 ? 9 : (wmax + 1 <= 17 ? 17 : 33);
+  return (size_t)n_heads * ((size_t)(nv - 1) * (nv - 1) + (nv - 1)) * sizeof(double);
+}
+
+cudaError_t launch_predict(const PredictArgs& args, cudaStream_t s) {
+  // The mean over the windows does not depend on their order: sort them widest
+  // first, so that windows whose widths are powers of two and add up to at most
+  // 32 lanes each start at a multiple of their width.
+  PredictArgs a = args;
+  if (a.mode != kPredFull && !predict_factor_eligible(a)) {
+    if (a.mode == kPredFactor) return cudaSuccess;   // nothing to precompute
+    a.mode = kPredFull;
+  }
+  sort_windows(a);
   return a.head_dim == 64 ? launch_d<64>(a, s) : launch_d<128>(a, s);
 }
 

@@ -60,9 +60,10 @@ int main(void) {
          offsetof(asp_kv, page_table), offsetof(asp_kv, seq_lens));
   printf("asp_pred_cfg %zu %zu %zu %zu\n", sizeof(asp_pred_cfg), offsetof(asp_pred_cfg, windows), offsetof(asp_pred_cfg, lambda),
          offsetof(asp_pred_cfg, pool));
-  printf("asp_decode_args %zu %zu %zu %zu %zu %zu %zu\n", sizeof(asp_decode_args), offsetof(asp_decode_args, kv),
+  printf("asp_decode_args %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(asp_decode_args), offsetof(asp_decode_args, kv),
          offsetof(asp_decode_args, workspace_bytes), offsetof(asp_decode_args, s_main), offsetof(asp_decode_args, timing),
-         offsetof(asp_decode_args, k_new), offsetof(asp_decode_args, quest_page));
+         offsetof(asp_decode_args, k_new), offsetof(asp_decode_args, quest_page), offsetof(asp_decode_args, pred_factor_cur),
+         offsetof(asp_decode_args, pred_factor_valid), offsetof(asp_decode_args, pred_factor_next));
   return 0;
 }
 '''
@@ -78,11 +79,12 @@ int main(void) {
     assert lines["asp_kv"] == [ctypes.sizeof(K), K.k.offset, K.page_size.offset, K.page_table.offset, K.seq_lens.offset]
     assert lines["asp_pred_cfg"] == [ctypes.sizeof(P), P.windows.offset, P.lam.offset, P.pool.offset]
     assert lines["asp_decode_args"] == [ctypes.sizeof(D), D.kv.offset, D.workspace_bytes.offset, D.s_main.offset,
-                                        D.timing.offset, D.k_new.offset, D.quest_page.offset]
+                                        D.timing.offset, D.k_new.offset, D.quest_page.offset, D.pred_factor_cur.offset,
+                                        D.pred_factor_valid.offset, D.pred_factor_next.offset]
 
 
 def test_version_and_status_strings(lib):
-    assert lib.asp_abi_version() == 3
+    assert lib.asp_abi_version() == 4
     assert L.status_string(L.ASP_OK) == "ok"
     assert "workspace" in L.status_string(L.ASP_ERR_WORKSPACE)
     assert L.status_string(99) == "unknown status"
@@ -255,6 +257,17 @@ def test_predict_rejects_shapes(lib):
     assert lib.asp_predict_query(None, 0, None, 0, 2, 8, 128, ctypes.byref(cfg), FAKE, None) == L.ASP_ERR_INVALID_ARG
     assert lib.asp_predict_query(FAKE, 0, None, 0, 2, 8, 128, None, FAKE, None) == L.ASP_ERR_INVALID_ARG
     assert lib.asp_predict_query(FAKE, 0, FAKE, 9, 2, 8, 128, ctypes.byref(cfg), FAKE, None) == L.ASP_ERR_INVALID_ARG
+
+
+def test_predictor_factor_bytes(lib):
+    """One fp64 factor per query head: the widest window's scaled rows and inverse diagonal."""
+    cfg = L.PredCfg(16, (4, 8, 16), 1e-2)
+    assert lib.asp_pred_factor_bytes(8, 32, ctypes.byref(cfg.struct)) == 8 * 32 * (16 * 16 + 16) * 8
+    cfg8 = L.PredCfg(16, (4, 8), 1e-2)
+    assert lib.asp_pred_factor_bytes(2, 4, ctypes.byref(cfg8.struct)) == 2 * 4 * (8 * 8 + 8) * 8
+    assert lib.asp_pred_factor_bytes(0, 32, ctypes.byref(cfg.struct)) == 0
+    bad = L.PredCfg(4, (8,), 1e-2)   # a window wider than the history
+    assert lib.asp_pred_factor_bytes(8, 32, ctypes.byref(bad.struct)) == 0
 
 
 def test_decode_step_and_wait_validation(lib):

@@ -228,6 +228,54 @@ def test_decode_selection_ties_across_the_halves_of_a_row():
     assert np.array_equal(idx, ref_idx)
 
 
+@pytest.mark.parametrize("precompute", [True, False], ids=["factor_from_previous_step", "full_factorisation"])
+def test_predictor_over_several_steps_against_the_oracle(precompute):
+    """Four decode steps at the Qwen3-8B head shapes (W = 16, windows 4, 8, 16).  With
+    the precomputation every step after the first predicts with the lag factor the
+    step before it stored (the next step's lag Gram holds q_t and the 15 queries
+    before it): the stored factor equals the Cholesky factor of that Gram computed
+    on the host, and every step's prediction matches the oracle's on the ring's
+    history, as it does with the full factorisation in every step."""
+    B, Hkv, G, d, T, C, W, windows, lam = 8, 8, 4, 128, 4096, 256, 16, (4, 8, 16), 1e-2
+    Hq = Hkv * G
+    g = torch.Generator().manual_seed(31)
+    k = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).to(DEV)
+    v = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).to(DEV)
+    kv = asp.KV(k, v, torch.full((B,), T, dtype=torch.int32, device=DEV), t_max=T)
+    seq = [torch.randn(B, Hq, d, generator=g)]
+    for _ in range(W + 4):
+        seq.append(0.9 * seq[-1] + 0.1 * torch.randn(B, Hq, d, generator=g))
+    seq = [x.to(torch.bfloat16).float() for x in seq]   # the queries arrive as bf16
+    hist = torch.stack(seq[:W + 1], dim=2)              # oldest first, ring_start 0
+    st = asp.DecodeState(kv, Hq, asp.PredCfg(W, windows, lam), C, hist.to(DEV).contiguous(),
+                         precompute_factor=precompute)
+    assert (st.pred_factor is not None) == precompute
+    idx0, cnt0 = synth.random_selection(B, Hkv, C, [T] * B, seed=3)
+    st.set_selection(idx0.to(DEV), cnt0.to(DEV))
+    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=DEV)
+    for step in range(4):
+        t = W + 1 + step                                 # seq[t] is this step's query
+        nxt = 1 - st.cur
+        st.step(seq[t].to(torch.bfloat16).to(DEV), out)
+        assert asp.wait_selection(st.ev_sel_done, 60_000_000) == 0
+        torch.cuda.synchronize()
+        window = torch.stack(seq[t - W:t + 1], dim=2)    # q_{t-W} .. q_t
+        ref = oracle.predict_query(window.double().numpy(), windows, lam)
+        assert_pred_close(st.qpred.cpu().numpy(), ref, f"step {step}")
+        if precompute:
+            # the factor stored for the next step: its lags are q_t, q_{t-1}, ... (newest first)
+            lags = torch.stack([seq[t - r] for r in range(W)], dim=2).double()      # [B, Hq, W, d]
+            gram = lags @ lags.transpose(-1, -2) + lam * torch.eye(W, dtype=torch.float64)
+            L = torch.linalg.cholesky(gram)
+            inv = 1.0 / torch.diagonal(L, dim1=-2, dim2=-1)
+            scaled = torch.tril(L * inv[..., :, None], diagonal=-1)
+            fac = st.pred_factor[nxt].cpu().view(B * Hq, W * W + W)
+            got_rows = torch.tril(fac[:, :W * W].view(B * Hq, W, W), diagonal=-1)
+            assert torch.allclose(got_rows, scaled.view(B * Hq, W, W), rtol=1e-4, atol=1e-5), f"step {step} factor"
+            assert torch.allclose(fac[:, W * W:], inv.view(B * Hq, W), rtol=1e-4), f"step {step} 1/diag"
+    assert asp.device_status() == 0
+
+
 def test_decode_selection_up_to_32k_tokens_matches_the_oracle_on_ragged_rows():
     """Rows of at most 32K tokens keep the whole row in registers (one 16-byte vector
     per lane and chunk): ragged lengths that end inside a vector, inside a warp's
