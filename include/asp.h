@@ -250,7 +250,7 @@ ASP_API size_t asp_pred_factor_bytes(int batch, int n_q_heads, const asp_pred_cf
  * ASP_NOALLOC_SCRATCH_BYTES bytes (2 MiB), that every GPU which loads the library
  * holds until the process exits.  Sizes whose partials would not fit (compare
  * asp_attend_workspace_bytes) return ASP_ERR_WORKSPACE and enqueue nothing; with
- * the current split plan the partials stay below 1.3 MB for every valid size.
+ * the current split plan the partials stay below 1.9 MB for every valid size.
  * The first call on a device looks up the array's device address on that device
  * (the device must be current); make that first call before any stream capture.
  * All calls share the one array and it keeps the last call's contents; nothing in

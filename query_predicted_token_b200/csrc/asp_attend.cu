@@ -429,7 +429,7 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
 // their accumulators are not kept.  a0: (row g, k 2t..2t+1), a2: (row g, k
 // 8+2t..9+2t); b0: (k 2t..2t+1, col g), b1: (k 8+2t..9+2t, col g).
 __device__ __forceinline__ void mma_top8(float& d0, float& d1, uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-  float x2, x3;
+  [[maybe_unused]] float x2, x3;   // rows 8-15: zero, discarded
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%10, %11, %12, %13};"
@@ -470,6 +470,9 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
     mbar_init_fence();
   }
   __syncwarp();
+  // launched with programmatic stream serialisation: everything above overlaps the
+  // previous kernel; every global access comes after its completion
+  pdl_wait();
 
   // A persistent grid: each CTA takes work items (unit, split) in turn; the stage
   // barriers' phases run on over the items (tbase: this warp's tiles so far).
@@ -495,7 +498,6 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
   const int r0 = split * p.rows_per_split;
   const int r1 = min(n_rows, r0 + p.rows_per_split);
   const int n_tiles = r1 > r0 ? (r1 - r0 + kTile - 1) / kTile : 0;
-  const int32_t* idx_row = n_sel ? p.idx + (size_t)unit * p.C : nullptr;
 
   // query fragments: head g (zero rows for g >= G), channels 16kk + 2t (+8)
   uint32_t qa[KS][2];
@@ -515,8 +517,17 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
     const uint8_t* src;
     bool valid;
   };
-  // Row source of this lane for tile t (lanes 0-15: K rows, 16-31: V rows).
-  auto resolve = [&](int tt) -> RowSrc {
+  // The raw index of this lane's row in tile t, loaded without waiting for the
+  // unit's count (any r < C lies inside the index array): the index loads of a
+  // tile go out a tile ahead of its copies, and those of the first tiles together
+  // with the count.
+  auto load_raw = [&](int tt) -> int {
+    const int r = r0 + (warp + tt * kWarps) * kTile + (lane & 15);
+    return (p.idx && r < p.C) ? __ldg(p.idx + (size_t)unit * p.C + r) : 0;
+  };
+  // Row source of this lane for tile t (lanes 0-15: K rows, 16-31: V rows), given
+  // its raw index.
+  auto resolve = [&](int tt, int jraw) -> RowSrc {
     const int rr = lane & 15;
     const bool isv = lane >= 16;
     const int r = r0 + (warp + tt * kWarps) * kTile + rr;
@@ -524,7 +535,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
     int j = 0;
     if (valid) {
       if (r < n_sel) {
-        j = idx_row[r];
+        j = jraw;
         if (j < 0 || j >= T) {
           valid = false;
           if (!isv) flag_status(ASP_DEV_BAD_INDEX);
@@ -596,14 +607,19 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
   const uint32_t v_off = (uint32_t)(HALF + ((mat & 1) * 8 + mrow) * STRIDE + (mat >> 1) * 16);  // + 32 j
 
   uint32_t vmask[STAGES];
+  int raw[STAGES];
+#pragma unroll
+  for (int s = 0; s < STAGES; ++s) raw[s] = load_raw(s);
   int issued = 0;
-#pragma unroll 1
-  for (int s = 0; s < STAGES && s < my_tiles; ++s) {
-    const int sl = (int)((tbase + s) % STAGES);
-    vmask[sl] = issue(resolve(s), sl);
-    ++issued;
+#pragma unroll
+  for (int s = 0; s < STAGES; ++s) {
+    if (s < my_tiles) {
+      const int sl = (int)((tbase + s) % STAGES);
+      vmask[sl] = issue(resolve(s, raw[s]), sl);
+      ++issued;
+    }
   }
-  RowSrc next = issued < my_tiles ? resolve(issued) : RowSrc{nullptr, false};
+  int raw_next = issued < my_tiles ? load_raw(issued) : 0;
 
   int consumed = 0;
   bool ok = true;
@@ -669,9 +685,9 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
     }
     __syncwarp();
     if (issued < my_tiles) {
-      vmask[slot] = issue(next, slot);
+      vmask[slot] = issue(resolve(issued, raw_next), slot);
       ++issued;
-      if (issued < my_tiles) next = resolve(issued);
+      if (issued < my_tiles) raw_next = load_raw(issued);
     }
   }
   if (!ok) {
@@ -1174,7 +1190,8 @@ __global__ void __launch_bounds__(D) attend_merge_kernel(const float* __restrict
   using E = Elem<KT>;
   const size_t bh = blockIdx.x;
   const int c = threadIdx.x;
-  pdl_wait();   // the split partials come from the previous kernel
+  pdl_trigger();   // the next call's attention may start its prologue
+  pdl_wait();      // the split partials come from the previous kernel
   const float* ml = part_ml + bh * splits * 2;
   float M = -INFINITY;
   for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[2 * s]);
@@ -1218,8 +1235,7 @@ cudaError_t launch_mma(const AttParams& p, cudaStream_t s) {
   const size_t merge = (size_t)kWarps * G * (D + 2) * 4;
   if (smem < merge) smem = merge;
   if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
-  kern<<<dim3(p.ctas), kWarps * 32, smem, s>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(kern, dim3(p.ctas), dim3(kWarps * 32), smem, s, p);
   if (e != cudaSuccess || p.splits == 1) return e;
   return launch_pdl(attend_merge_kernel<__nv_bfloat16, D>, dim3(p.batch * p.n_q_heads), dim3(D), 0, s,
                     (const float*)p.part_o, (const float*)p.part_ml, p.splits, p.out, p.lse);
@@ -1250,9 +1266,9 @@ cudaError_t dispatch_g(int G, const AttParams& p, cudaStream_t s) {
 }  // namespace
 
 // Split plan of the per-item kernels: as many splits per KV head as fit in one
-// wave of resident CTAs on a 148-SM B200 (by default 3 CTAs per SM for G <= 4, 2
-// for G = 8, set by the registers), each split a multiple of 64 rows (one 16-row
-// tile per warp).  The gather kernel's plan (stand-alone calls; the decode step
+// wave of resident CTAs on a 148-SM B200 (by default 3 CTAs per SM: 166 registers
+// x 128 threads; 2 per SM at G = 8 measured 41 against 36.5 us on the Qwen3-32B
+// shapes), each split a multiple of 64 rows (one 16-row tile per warp).  The gather kernel's plan (stand-alone calls; the decode step
 // keeps the per-item kernel, whose CTA fits beside the key scan's): every unit
 // planned for C + max_tail rows, its tiles spread evenly over at most one CTA per
 // SM (and at least 8 tiles per CTA), partials in 2 slots per CTA when a unit is
@@ -1288,7 +1304,7 @@ AttendPlan attend_plan(int batch, int n_q_heads, int n_kv_heads, int head_dim, i
   const long units = (long)batch * n_kv_heads;
   if (rows <= 0 || units <= 0 || n_kv_heads <= 0) return pl;
   const int G = n_q_heads / n_kv_heads;
-  const long target = 148L * (ctas_per_sm > 0 ? ctas_per_sm : (G >= 8 ? 2 : 3));
+  const long target = 148L * (ctas_per_sm > 0 ? ctas_per_sm : 3);
   const int quantum = kTile * kWarps;
   long splits = target / units;
   if (splits < 1) splits = 1;

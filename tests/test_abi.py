@@ -173,7 +173,7 @@ def _ring_ws(B, Hq, Hkv, d, C, max_tail):
 def _split_ws(B, Hq, Hkv, d, C, max_tail, ctas_per_sm):
     # the per-item kernels: splits of a multiple of 64 rows filling one wave
     units, G = B * Hkv, Hq // Hkv
-    target = 148 * (ctas_per_sm or (2 if G >= 8 else 3))
+    target = 148 * (ctas_per_sm or 3)
     splits = max(1, target // units)
     rows = C + max_tail
     per = -(-(-(-rows // splits)) // 64) * 64
