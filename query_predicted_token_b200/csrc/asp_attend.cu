@@ -446,11 +446,28 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, u
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
+// Cluster helpers: a barrier over the CTAs of the cluster (release / acquire, so
+// that shared-memory stores before it are seen after it), and a store of one
+// float into the shared memory of CTA `rank` of the cluster at the offset of `p`.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void st_cluster_f32(const float* p, uint32_t rank, float v) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+
 // LEAN: the row copies are issued from a partly unrolled loop, which keeps the
 // registers at the level that lets one CTA share an SM with the key scan's and the
 // predictor's (the decode step); the fully unrolled form keeps more copies in
 // flight where three CTAs share an SM (stand-alone calls).
-template <int D, int G, int STAGES, bool LEAN>
+// CLUSTER: one work item per CTA and the splits of a unit form one thread-block
+// cluster (rank = split): the splits' partials meet in the shared memory of the
+// cluster's first CTA, which merges them and writes the output -- no partials in
+// global memory and no merge kernel.
+template <int D, int G, int STAGES, bool LEAN, bool CLUSTER = false>
 __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
   constexpr int ROW_BYTES = D * 2;
   constexpr int STRIDE = ROW_BYTES + 16;          // padded row pitch in shared memory
@@ -711,6 +728,9 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
     }
   }
   __syncthreads();
+  // cluster: every CTA of the cluster is past its stages, so the first CTA's
+  // shared memory beyond its warp-merge area is free for the partials
+  if constexpr (CLUSTER) cluster_sync_all();
   for (int e = threadIdx.x; e < G * D; e += kWarps * 32) {
     const int gg = e / D, c = e - gg * D;
     float M = -INFINITY;
@@ -728,7 +748,17 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
       }
     }
     const size_t bh = (size_t)b * p.n_q_heads + h * G + gg;
-    if (p.splits == 1) {
+    if constexpr (CLUSTER) {
+      // the first CTA's partial slots, after its warp-merge area: [splits][G][D]
+      // outputs, then [splits][G][2] (max, sum)
+      float* slot_o = mml + kWarps * G * 2;
+      float* slot_ml = slot_o + p.splits * G * D;
+      st_cluster_f32(slot_o + (split * G + gg) * D + c, 0, O);
+      if (c == 0) {
+        st_cluster_f32(slot_ml + (split * G + gg) * 2 + 0, 0, M);
+        st_cluster_f32(slot_ml + (split * G + gg) * 2 + 1, 0, L);
+      }
+    } else if (p.splits == 1) {
       const float r = L > 0.f ? O / L : 0.f;
       static_cast<__nv_bfloat16*>(p.out)[bh * D + c] = __float2bfloat16_rn(r);
       if (c == 0 && p.lse) p.lse[bh] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
@@ -739,6 +769,32 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
         p.part_ml[(bh * p.splits + split) * 2 + 1] = L;
       }
     }
+  }
+  if constexpr (CLUSTER) {
+    cluster_sync_all();   // the partials are in the first CTA's shared memory
+    if (split == 0) {
+      const float* slot_o = mml + kWarps * G * 2;
+      const float* slot_ml = slot_o + p.splits * G * D;
+      for (int e = threadIdx.x; e < G * D; e += kWarps * 32) {
+        const int gg = e / D, c = e - gg * D;
+        float M = -INFINITY;
+        for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, slot_ml[(sp * G + gg) * 2]);
+        float L = 0.f, O = 0.f;
+        if (M != -INFINITY) {
+          for (int sp = 0; sp < p.splits; ++sp) {
+            const float ms = slot_ml[(sp * G + gg) * 2];
+            if (ms == -INFINITY) continue;
+            const float f = ex2(ms - M);
+            L += slot_ml[(sp * G + gg) * 2 + 1] * f;
+            O += slot_o[(sp * G + gg) * D + c] * f;
+          }
+        }
+        const size_t bh = (size_t)b * p.n_q_heads + h * G + gg;
+        static_cast<__nv_bfloat16*>(p.out)[bh * D + c] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
+        if (c == 0 && p.lse) p.lse[bh] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+      }
+    }
+    break;   // one item per CTA
   }
   // the next item's copies overwrite the merge area: generic accesses first
   fence_proxy_async_smem();
@@ -1230,10 +1286,22 @@ template <int D, int G>
 cudaError_t launch_mma(const AttParams& p, cudaStream_t s) {
   constexpr int STAGES = 2;
   constexpr int TILE_BYTES = 2 * kTile * (D * 2 + 16);
-  auto kern = p.lean ? attend_mma_kernel<D, G, STAGES, true> : attend_mma_kernel<D, G, STAGES, false>;
   size_t smem = (size_t)kWarps * STAGES * TILE_BYTES + kWarps * STAGES * 8;
   const size_t merge = (size_t)kWarps * G * (D + 2) * 4;
   if (smem < merge) smem = merge;
+  // One item per CTA and 4 to 8 splits (a portable cluster), whose partials fit
+  // beside the warp-merge area: the splits merge inside their cluster.  Measured
+  // alone (back to back over copies of the cache): 6 splits (Qwen3-8B shapes)
+  // 19.8 against 22.3 us with the merge kernel; 3 splits (Qwen3-32B shapes) 34.8
+  // against 33.5 us, so fewer splits keep the merge kernel.  Letting the next
+  // kernel launch early from the cluster kernel cost 9 us at 3 splits.
+  if (!p.lean && p.splits >= 4 && p.splits <= 8 && p.ctas == p.n_items &&
+      merge + (size_t)p.splits * G * (D + 2) * 4 <= smem) {
+    auto kc = attend_mma_kernel<D, G, STAGES, false, true>;
+    if (prepare_kernel((const void*)kc, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
+    return launch_pdl_cluster(kc, dim3(p.ctas), dim3(kWarps * 32), smem, s, p.splits, p);
+  }
+  auto kern = p.lean ? attend_mma_kernel<D, G, STAGES, true> : attend_mma_kernel<D, G, STAGES, false>;
   if (prepare_kernel((const void*)kern, smem, kWarps * 32) < 1) return cudaErrorInvalidConfiguration;
   cudaError_t e = launch_pdl(kern, dim3(p.ctas), dim3(kWarps * 32), smem, s, p);
   if (e != cudaSuccess || p.splits == 1) return e;

@@ -43,6 +43,32 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// launch_pdl with thread-block clusters of `cluster_x` CTAs along x (grid.x a
+// multiple of it).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                               int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  int prio = 0;
+  if (cudaStreamGetPriority(s, &prio) != cudaSuccess) prio = 0;
+  cudaLaunchAttribute attr[3];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributePriority;
+  attr[1].val.priority = prio;
+  attr[2].id = cudaLaunchAttributeClusterDimension;
+  attr[2].val.clusterDim.x = (unsigned)cluster_x;
+  attr[2].val.clusterDim.y = 1;
+  attr[2].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 3;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // A plain launch (no early start) that carries the stream's priority like launch_pdl.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_prio(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {

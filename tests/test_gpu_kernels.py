@@ -329,6 +329,48 @@ def test_sparse_attend_gather_kernel(case):
     assert_lse_close(lse, ref_lse)
 
 
+def _standalone_splits(units, rows):
+    """Splits per unit of the per-item kernels' stand-alone plan (three 4-warp CTAs per
+    SM on 148 SMs, splits of a multiple of 64 rows)."""
+    splits = max(1, 444 // units)
+    per = -(-(-(-rows // splits)) // 64) * 64
+    return -(-rows // per)
+
+
+_CLUSTER_CASES = [
+    (8, 8, 4, 128, 2048, _lens(8, 2100, 3000, 4), 0, 0),
+    (55, 1, 8, 128, 2048, _lens(55, 2049, 2600, 5), 16, 0),
+    (37, 3, 2, 64, 1000, _lens(37, 900, 1400, 6), 0, 0),
+    (16, 4, 4, 128, 1024, _lens(16, 1100, 1500, 7), 0, 16),
+]
+
+
+@pytest.mark.parametrize("case", _CLUSTER_CASES, ids=["splits6_G4", "splits8_G8_paged", "splits4_d64_G2", "splits6_tail"])
+def test_sparse_attend_cluster_merge(case):
+    """bf16 attention whose stand-alone plan has 4 to 8 splits per unit: the splits of
+    a unit form one thread-block cluster and merge their partials in the first CTA's
+    shared memory.  Ragged rows (some units shorter than C), a paged cache, head
+    dimension 64 and a tail, against the oracle."""
+    B, Hkv, G, d, C, lens, page_size, tail = case
+    assert 4 <= _standalone_splits(B * Hkv, C + tail) <= 8
+    T = max(lens)
+    kvd, kv = make_cache(B, Hkv, d, T, torch.bfloat16, lens, page_size, seed=B + C + d)
+    tb = [max(0, t - tail) for t in lens]
+    idx, cnt = random_selection(B, Hkv, C, tb, seed=C + G + 1)
+    q = torch.randn(B, Hkv * G, d, generator=_gen(B * 5 + d)).to(torch.bfloat16).to(DEV)
+    out = torch.full((B, Hkv * G, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    lse = torch.full((B, Hkv * G), float("nan"), device=DEV)
+    ws = torch.empty(max(16, asp.attend_workspace_bytes(B, Hkv * G, Hkv, d, C, tail)), dtype=torch.uint8, device=DEV)
+    tail_begin = torch.tensor(tb, dtype=torch.int32, device=DEV) if tail else None
+    asp.sparse_attend(q, kv, idx.to(DEV), cnt.to(DEV), C, out, lse, tail_begin, tail, ws)
+    torch.cuda.synchronize()
+    keys, vals = host_sequences(kvd)
+    ref, ref_lse = oracle.sparse_attend(np64(q), [keys[b] for b in range(B)], [vals[b] for b in range(B)],
+                                        idx.numpy(), cnt.numpy(), tb if tail else None)
+    assert_out_close(out, ref, torch.bfloat16, f"cluster {case[:5]}")
+    assert_lse_close(lse, ref_lse)
+
+
 def test_gather_kernel_flags_out_of_range_indices_and_skips_them():
     B, Hkv, G, d, C, T = 64, 8, 2, 128, 1024, 1100
     kvd, kv = make_cache(B, Hkv, d, T, torch.bfloat16, [T] * B, seed=5)
