@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--layers", type=int, default=36,
                     help="also time a stack of this many layers (each with its own cache), steady-state period "
                          "(1: no stack)")
-    ap.add_argument("--profile", default=None, choices=["scan", "scan_cuda_cores", "attend", "page_scan"],
+    ap.add_argument("--profile", default=None, choices=["scan", "scan_cuda_cores", "attend", "page_scan", "decode"],
                     help="only build the workload and launch this kernel --steps times (for ncu captures); "
                          "prints no JSON line")
     ap.add_argument("--side-streams", type=int, default=1,
@@ -697,7 +697,8 @@ def profile_launches(args):
     each, for an ncu capture of that kernel alone (scan: the key scan as the library
     picks it; scan_cuda_cores: the CUDA-core scan on the same keys; attend: the
     sparse attention's stand-alone plan over a random selection; page_scan: the
-    page-bound scan of the page-level path)."""
+    page-bound scan of the page-level path; decode: whole decode steps, for the
+    selection or the predictor inside the step)."""
     import torch
     import query_predicted_token_b200 as asp
     import synth
@@ -713,7 +714,18 @@ def profile_launches(args):
     qpred = synth.query_history(wl, 1)[1][0].to(dev).contiguous()
     q = qpred.to(wl.torch_dtype())
     scores = torch.empty(B, Hkv, wl.t_max, device=dev)
-    if args.profile == "attend":
+    if args.profile == "decode":
+        qhist, q_next = synth.query_history(wl, steps=1)
+        st = asp.DecodeState(kv, Hq, asp.PredCfg(wl.W, wl.windows, wl.lam), C, qhist.to(dev).contiguous())
+        i0, c0 = synth.random_selection(B, Hkv, C, lens, seed=wl.seed + 99)
+        st.set_selection(i0.to(dev), c0.to(dev))
+        qt = q_next[0].to(wl.torch_dtype()).to(dev)
+        out = torch.empty(B, Hq, d, dtype=wl.torch_dtype(), device=dev)
+
+        def fn():
+            st.step(qt, out)
+            st.s_main.wait_event(st.ev_sel_done)
+    elif args.profile == "attend":
         idx, cnt = (x.to(dev) for x in synth.random_selection(B, Hkv, C, snap, seed=wl.seed + 99))
         tb = torch.tensor(snap, dtype=torch.int32, device=dev) if tail else None
         out = torch.empty(B, Hq, d, dtype=wl.torch_dtype(), device=dev)
