@@ -458,6 +458,13 @@ __device__ __forceinline__ void st_cluster_f32(const float* p, uint32_t rank, fl
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
 }
+// Four floats at a 16-byte aligned `p` into the shared memory of CTA `rank`.
+__device__ __forceinline__ void st_cluster_f32x4(const float* p, uint32_t rank, float4 v) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
 
 // LEAN: the row copies are issued from a partly unrolled loop, which keeps the
 // registers at the level that lets one CTA share an SM with the key scan's and the
@@ -728,9 +735,82 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
     }
   }
   __syncthreads();
-  // cluster: every CTA of the cluster is past its stages, so the first CTA's
-  // shared memory beyond its warp-merge area is free for the partials
-  if constexpr (CLUSTER) cluster_sync_all();
+  if constexpr (CLUSTER) {
+    // Every CTA of the cluster is past its stages, so the first CTA's shared memory
+    // beyond its warp-merge area is free for the partials: [splits][G][D] outputs,
+    // then [splits][G][2] (max, sum).  Four channels per thread and store.
+    cluster_sync_all();
+    float* slot_o = mml + kWarps * G * 2;   // 16-byte aligned: kWarps * G * (D + 2) floats in
+    float* slot_ml = slot_o + p.splits * G * D;
+    for (int e4 = threadIdx.x; e4 < G * D / 4; e4 += kWarps * 32) {
+      const int gg = (4 * e4) / D, c = 4 * e4 - gg * D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mml[(w * G + gg) * 2]);
+      float L = 0.f;
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+          const float mw = mml[(w * G + gg) * 2];
+          if (mw == -INFINITY) continue;
+          const float f = ex2(mw - M);
+          L += mml[(w * G + gg) * 2 + 1] * f;
+          const float4 x = *reinterpret_cast<const float4*>(mo + (w * G + gg) * D + c);
+          O.x += x.x * f;
+          O.y += x.y * f;
+          O.z += x.z * f;
+          O.w += x.w * f;
+        }
+      }
+      st_cluster_f32x4(slot_o + (split * G + gg) * D + c, 0, O);
+      if (c == 0) {
+        st_cluster_f32(slot_ml + (split * G + gg) * 2 + 0, 0, M);
+        st_cluster_f32(slot_ml + (split * G + gg) * 2 + 1, 0, L);
+      }
+    }
+    cluster_sync_all();   // the partials are in the first CTA's shared memory
+    if (split == 0) {
+      for (int e4 = threadIdx.x; e4 < G * D / 4; e4 += kWarps * 32) {
+        const int gg = (4 * e4) / D, c = 4 * e4 - gg * D;
+        float M = -INFINITY;
+        for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, slot_ml[(sp * G + gg) * 2]);
+        float L = 0.f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (M != -INFINITY) {
+          for (int sp = 0; sp < p.splits; ++sp) {
+            const float ms = slot_ml[(sp * G + gg) * 2];
+            if (ms == -INFINITY) continue;
+            const float f = ex2(ms - M);
+            L += slot_ml[(sp * G + gg) * 2 + 1] * f;
+            const float4 x = *reinterpret_cast<const float4*>(slot_o + (sp * G + gg) * D + c);
+            O.x += x.x * f;
+            O.y += x.y * f;
+            O.z += x.z * f;
+            O.w += x.w * f;
+          }
+        }
+        const float r = L > 0.f ? 1.f / L : 0.f;
+        const size_t bh = (size_t)b * p.n_q_heads + h * G + gg;
+        const __nv_bfloat162 lo2 = __floats2bfloat162_rn(O.x * r, O.y * r);
+        const __nv_bfloat162 hi2 = __floats2bfloat162_rn(O.z * r, O.w * r);
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + bh * D + c;
+        if ((reinterpret_cast<uintptr_t>(p.out) & 7) == 0) {   // D * 2 and c * 2 keep the 8-byte alignment
+          uint2 packed;
+          packed.x = *reinterpret_cast<const uint32_t*>(&lo2);
+          packed.y = *reinterpret_cast<const uint32_t*>(&hi2);
+          *reinterpret_cast<uint2*>(dst) = packed;
+        } else {
+          dst[0] = lo2.x;
+          dst[1] = lo2.y;
+          dst[2] = hi2.x;
+          dst[3] = hi2.y;
+        }
+        if (c == 0 && p.lse) p.lse[bh] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+      }
+    }
+    break;   // one item per CTA
+  } else {
   for (int e = threadIdx.x; e < G * D; e += kWarps * 32) {
     const int gg = e / D, c = e - gg * D;
     float M = -INFINITY;
@@ -748,17 +828,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
       }
     }
     const size_t bh = (size_t)b * p.n_q_heads + h * G + gg;
-    if constexpr (CLUSTER) {
-      // the first CTA's partial slots, after its warp-merge area: [splits][G][D]
-      // outputs, then [splits][G][2] (max, sum)
-      float* slot_o = mml + kWarps * G * 2;
-      float* slot_ml = slot_o + p.splits * G * D;
-      st_cluster_f32(slot_o + (split * G + gg) * D + c, 0, O);
-      if (c == 0) {
-        st_cluster_f32(slot_ml + (split * G + gg) * 2 + 0, 0, M);
-        st_cluster_f32(slot_ml + (split * G + gg) * 2 + 1, 0, L);
-      }
-    } else if (p.splits == 1) {
+    if (p.splits == 1) {
       const float r = L > 0.f ? O / L : 0.f;
       static_cast<__nv_bfloat16*>(p.out)[bh * D + c] = __float2bfloat16_rn(r);
       if (c == 0 && p.lse) p.lse[bh] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
@@ -770,31 +840,6 @@ __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
       }
     }
   }
-  if constexpr (CLUSTER) {
-    cluster_sync_all();   // the partials are in the first CTA's shared memory
-    if (split == 0) {
-      const float* slot_o = mml + kWarps * G * 2;
-      const float* slot_ml = slot_o + p.splits * G * D;
-      for (int e = threadIdx.x; e < G * D; e += kWarps * 32) {
-        const int gg = e / D, c = e - gg * D;
-        float M = -INFINITY;
-        for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, slot_ml[(sp * G + gg) * 2]);
-        float L = 0.f, O = 0.f;
-        if (M != -INFINITY) {
-          for (int sp = 0; sp < p.splits; ++sp) {
-            const float ms = slot_ml[(sp * G + gg) * 2];
-            if (ms == -INFINITY) continue;
-            const float f = ex2(ms - M);
-            L += slot_ml[(sp * G + gg) * 2 + 1] * f;
-            O += slot_o[(sp * G + gg) * D + c] * f;
-          }
-        }
-        const size_t bh = (size_t)b * p.n_q_heads + h * G + gg;
-        static_cast<__nv_bfloat16*>(p.out)[bh * D + c] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
-        if (c == 0 && p.lse) p.lse[bh] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
-      }
-    }
-    break;   // one item per CTA
   }
   // the next item's copies overwrite the merge area: generic accesses first
   fence_proxy_async_smem();
