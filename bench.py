@@ -456,10 +456,14 @@ def decode_record(wl, dev, args, flush, peak, peak_kind, *, headline, group=None
     assert asp.device_status() == 0
 
     # the stand-alone plan runs the persistent gather kernel from 200 16-row tiles per SM up
-    # (148 SMs, C + tail rows a unit, a tail of at most max(C, 4096)), the per-item kernel otherwise
+    # (148 SMs, C + tail rows a unit, a tail of at most max(C, 4096)), the per-item kernel otherwise:
+    # three 4-warp CTAs per SM, splits of a multiple of 64 rows, merged inside a thread-block
+    # cluster when there are 4 to 8 of them, else by the merge kernel
     att_tiles = B * Hkv * ((C + tail + 15) // 16)
-    att_kernel = ("attend_gather_kernel" if att_tiles >= 200 * 148 and tail <= max(C, 4096)
-                  else "attend_mma_kernel")
+    att_splits = -(-(C + tail) // (-(-(-(-(C + tail) // max(1, 444 // (B * Hkv)))) // 64) * 64))
+    att_kernel = ("attend_gather_kernel (+ merge)" if att_tiles >= 200 * 148 and tail <= max(C, 4096)
+                  else "attend_mma_kernel (cluster merge)" if 4 <= att_splits <= 8
+                  else "attend_mma_kernel (+ merge)")
     step_us = statistics.mean(step_ms) * 1e3
     gbs = acct["total"] / (step_us / 1e6) / 1e9
     traffic = read_traffic("asp_score_tc.cu", 1.0) if wl.name == "qwen3_8b_shaped_32k" else None
@@ -481,7 +485,7 @@ def decode_record(wl, dev, args, flush, peak, peak_kind, *, headline, group=None
                                    rot_note.format(n=2, what="keys") + "; cold: one launch after an L2 flush",
                                    traffic=traffic,
                                    extra={"in_step_frac": round(acct["score"] / (statistics.mean(kern_ms["score"]) / 1e3) / 1e9 / peak, 4)}),
-        "roofline_attend": roofline_entry(att_kernel + " (+ merge) (sparse attention, stand-alone plan)",
+        "roofline_attend": roofline_entry(att_kernel + " (sparse attention, stand-alone plan)",
                                           att_bytes, att_rot, att_cold, peak, peak_kind,
                                           rot_note.format(n=R, what="K/V cache") + "; cold: one launch after an L2 flush"),
     }
