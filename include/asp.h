@@ -138,8 +138,9 @@ typedef struct {
  * window).  For each query head and each window w: ridge-fit q_t on the lags
  * q_{t-w}..q_{t-1} over the head_dim channels, a = (X X^T + lambda I)^-1 X q_t,
  * turn a into weights (softmax or raw), apply weight i to q_{t-w+i}; average
- * the window predictions.  The Gram matrix and right-hand side are formed in fp32;
- * the Cholesky factorisation, both substitutions and the weights run in fp64.
+ * the window predictions.  The Gram matrix and right-hand side are formed in fp32,
+ * the Cholesky factorisation and both substitutions run in fp64, the softmax of
+ * the coefficients in fp32.
  *
  * qhist : device fp32 ring [batch, n_q_heads, W+1, head_dim].  Slot
  *         (ring_start + s) % (W+1) holds the s-th oldest vector (s = 0..W).
