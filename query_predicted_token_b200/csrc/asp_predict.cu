@@ -181,17 +181,26 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
       }
     }
   }
+  constexpr int WMAX = NV - 1;   // lags the registers can hold
+  // the stored factor of one head: rows of L scaled by 1 / L_ii ([WMAX][WMAX], j < i),
+  // then the 1 / L_ii ([WMAX]); lane i's row is requested with the history, so
+  // that both loads share one round trip
+  constexpr int kFac = WMAX * WMAX + WMAX;
+  double srow[MODE == kPredUsing ? WMAX : 1];
+  double my_inv_f = 0.0;
+  if constexpr (MODE == kPredUsing) {
+    const double* fac = a.factor_in + (size_t)head * kFac;
+#pragma unroll
+    for (int j = 0; j < WMAX; ++j) srow[j] = (lane < WMAX && j < lane) ? fac[lane * WMAX + j] : 0.0;
+    my_inv_f = lane < WMAX ? fac[WMAX * WMAX + lane] : 0.0;
+  }
   if (MODE != kPredFactor && a.q_new) {   // push q_t into the ring: it replaces the oldest slot (ring_start)
     float* dst = hist + (size_t)a.ring_start * D + lane * CPL;
 #pragma unroll
     for (int c = 0; c < CPL; ++c) dst[c] = h[0][c];
   }
 
-  constexpr int WMAX = NV - 1;   // lags the registers can hold
   const int wm = wmax;
-  // the stored factor of one head: rows of L scaled by 1 / L_ii ([WMAX][WMAX], j < i),
-  // then the 1 / L_ii ([WMAX])
-  constexpr int kFac = WMAX * WMAX + WMAX;
   if constexpr (MODE == kPredUsing) {
     // right-hand side only: the lags' dot products with the target, reduced over
     // the warp (lane r then holds rhs_r)
@@ -209,11 +218,7 @@ __global__ void __launch_bounds__(kWarps * 32, NV <= 17 ? 4 : 1) predict_kernel(
     ReduceScatter<32, 16>::run(part, lane);
     // forward substitution L z = rhs with the stored factor: z_i = rhs_i / L_ii -
     // sum_{j<i} (L_ij / L_ii) z_j, one shuffle and one multiply-add per step
-    const double* fac = a.factor_in + (size_t)head * kFac;
-    double srow[WMAX];
-#pragma unroll
-    for (int j = 0; j < WMAX; ++j) srow[j] = (lane < WMAX && j < lane) ? fac[lane * WMAX + j] : 0.0;
-    const double my_inv = lane < WMAX ? fac[WMAX * WMAX + lane] : 0.0;
+    const double my_inv = my_inv_f;
     double zacc = lane < WMAX ? (double)part[0] * my_inv : 0.0;
 #pragma unroll
     for (int k = 0; k < WMAX; ++k) {
