@@ -3,7 +3,10 @@
 // The C largest scores of scores[0:T_b] (IEEE order, -0.0 == +0.0), ties at the
 // threshold to the lowest index, written ascending.
 //
-// One 1024-thread CTA per row.  The row's 32-bit order keys live in shared
+// Two kernels, one 1024-thread CTA per row in both.  select_regs_kernel (the
+// decode step's rows of up to 32K tokens, the first digit's histogram given by
+// the key scan) is described at its definition below.  select_kernel serves
+// longer rows and stand-alone calls: the row's 32-bit order keys live in shared
 // memory (up to 48K keys; longer rows are re-read from L2 in every sweep), so
 // no step needs another CTA.  When the first digit's histogram is given, the
 // threshold digit is found while the row's scores are still loading, and every
