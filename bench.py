@@ -825,9 +825,16 @@ def main():
             stack["page_level_period_us_from_one_layer"] = round(extra["page_level"]["step_us"] * stack["layers"], 1)
             stack["full_attention_period_us_from_one_layer"] = round(
                 extra["full_attention"]["step_us"] * stack["layers"], 1)
-        # the decode step's attention launches a merge when its plan splits the rows
+        # the decode step's attention launches a merge when its plan splits the rows,
+        # and the step launches the next step's lag factorisation when the selection's
+        # CTAs (one per row) and the factorisation's (one per 4 query heads) fit on the
+        # SMs together, for windows that are powers of two filling at most 32 lags
         dec_ws = int(asp.lib().asp_decode_workspace_bytes(B, Hq, Hkv, d, C, 0))
         splits = dec_ws > B * Hkv * 2048 * 4
+        win = sorted(wl.windows)
+        nv = 9 if max(win) + 1 <= 9 else (17 if max(win) + 1 <= 17 else 33)
+        factor = (all(w & (w - 1) == 0 for w in win) and sum(win) <= 32 and max(win) == nv - 1 and
+                  B * Hkv + -(-B * Hq // 4) <= torch.cuda.get_device_properties(0).multi_processor_count)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": round(ms_per_step, 4),
@@ -843,7 +850,7 @@ def main():
             "clocks": clocks.summary(),
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": io[0],
                     "d2h_bytes_per_step": io[1]},
-            "gpu_launches": args.steps * (4 + (1 if splits else 0)),
+            "gpu_launches": args.steps * (4 + (1 if splits else 0) + (1 if factor else 0)),
             "cpu_baseline": cpu,
             "workloads": subs or None,
             "comparison": {"full_attention": extra.get("full_attention"),
