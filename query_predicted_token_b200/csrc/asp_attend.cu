@@ -473,7 +473,9 @@ __device__ __forceinline__ void st_cluster_f32x4(const float* p, uint32_t rank, 
 // CLUSTER: one work item per CTA and the splits of a unit form one thread-block
 // cluster (rank = split): the splits' partials meet in the shared memory of the
 // cluster's first CTA, which merges them and writes the output -- no partials in
-// global memory and no merge kernel.
+// global memory and no merge kernel.  Every CTA reaches both cluster barriers:
+// the only waits before them are the bounded stage waits, and no CTA leaves the
+// item loop early in this mode.
 template <int D, int G, int STAGES, bool LEAN, bool CLUSTER = false>
 __global__ void __launch_bounds__(kWarps * 32) attend_mma_kernel(AttParams p) {
   constexpr int ROW_BYTES = D * 2;

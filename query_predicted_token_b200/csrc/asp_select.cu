@@ -607,7 +607,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_regs_kernel(SelectArgs a) 
   const float lo0 = key_edge(prefix), hi0 = edge_above(prefix, kTopShift);
 
   const bool landed = mbar_wait(&s_bar, 0);
-  if (!__syncthreads_and(landed)) return;   // ASP_DEV_WAIT_LIMIT recorded
+  if (!__syncthreads_and(landed)) {   // ASP_DEV_WAIT_LIMIT recorded
+    mbar_wait(&s_bar, 0);   // give the row's copies one more bounded wait before leaving
+    return;
+  }
 
   // ---- the one pass over the row: bit 4k + c of gk / ck is the unit of vector
   // (k + lane) mod 8, element c; a rotation by 4 (lane mod 8) puts the bits in index
