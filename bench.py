@@ -368,6 +368,8 @@ def decode_record(wl, dev, args, flush, peak, peak_kind, *, headline, group=None
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     acct = step_bytes(wl, lens)
 
+    copy_stream = torch.cuda.Stream(device=dev)
+
     def one_step(state, k=None, e2e=False):
         with torch.cuda.stream(s_main):
             flush.zero_()                                   # L2 flush, outside the timed events
@@ -377,7 +379,10 @@ def decode_record(wl, dev, args, flush, peak, peak_kind, *, headline, group=None
                 q_t.copy_(q_host, non_blocking=True)
             state.step(q_t, out, lse)
             if e2e:   # the output is ready when the attention ends: read it back while the selection runs
-                out_host.copy_(out, non_blocking=True)
+                copy_stream.wait_event(state.ev_attend_done)
+                with torch.cuda.stream(copy_stream):
+                    out_host.copy_(out, non_blocking=True)
+                s_main.wait_stream(copy_stream)
             s_main.wait_event(state.ev_sel_done)
             if k is not None:
                 ev[k][1].record(s_main)

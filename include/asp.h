@@ -48,7 +48,7 @@
 extern "C" {
 #endif
 
-#define ASP_ABI_VERSION 4
+#define ASP_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define ASP_API __attribute__((visibility("default")))
@@ -355,6 +355,11 @@ typedef struct {
   double* pred_factor_cur;
   int pred_factor_valid;
   double* pred_factor_next;
+  /* Optional: recorded on s_main as soon as this step's out and lse are written
+   * (before the main stream's later work of the step, such as the factorisation),
+   * so that a caller can copy the output back while the selection still runs.
+   * NULL: not recorded. */
+  asp_event_t ev_attend_done;
 } asp_decode_args;
 
 ASP_API asp_status asp_decode_step(const asp_decode_args* args);

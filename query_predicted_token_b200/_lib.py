@@ -44,7 +44,7 @@ class AspDecodeArgs(ctypes.Structure):
                 ("s_main", c_void_p), ("s_side", c_void_p), ("ev_fork", c_void_p), ("ev_sel_done", c_void_p),
                 ("timing", POINTER(c_void_p)), ("k_new", c_void_p), ("v_new", c_void_p), ("quest_meta", c_void_p),
                 ("quest_page", c_int), ("pred_factor_cur", c_void_p), ("pred_factor_valid", c_int),
-                ("pred_factor_next", c_void_p)]
+                ("pred_factor_next", c_void_p), ("ev_attend_done", c_void_p)]
 
 
 SIGNATURES = {
@@ -324,6 +324,8 @@ class DecodeState:
         self.s_side = s_side or torch.cuda.Stream(priority=-100)
         self.ev_fork = make_event()
         self.ev_sel_done = make_event()
+        # recorded when the step's output is written (a read-back may start there)
+        self.ev_attend_done = make_event()
         self.timing_events = [make_event(True) for _ in range(8)] if timing else None
         self._timing_arr = (c_void_p * 8)(*[event_handle(e) for e in self.timing_events]) if timing else None
 
@@ -353,6 +355,7 @@ class DecodeState:
         a.s_side = _stream(self.s_side)
         a.ev_fork = event_handle(self.ev_fork)
         a.ev_sel_done = event_handle(self.ev_sel_done)
+        a.ev_attend_done = event_handle(self.ev_attend_done)
         a.timing = ctypes.cast(self._timing_arr, POINTER(c_void_p)) if self._timing_arr is not None else None
         if self.pred_factor is not None:
             a.pred_factor_cur = _ptr(self.pred_factor[cur])
@@ -435,6 +438,7 @@ class DecodeState:
         # the events were last recorded inside the captures: record them once outside
         self.ev_fork.record(self.s_main)
         self.ev_sel_done.record(self.s_main)
+        self.ev_attend_done.record(self.s_main)
         self._graph_at = 0
         return n
 

@@ -384,6 +384,9 @@ asp_status asp_decode_step(const asp_decode_args* a) {
     e = asp::launch_attend(a->q_t, a->q_dtype == ASP_F32, a->n_q_heads, kv, a->idx_cur, a->count_cur, a->C,
                            a->tail_begin, a->max_tail, a->out, a->lse, a->workspace, plan, sm);
   if (e == cudaSuccess) e = mark(7, sm);
+  // out and lse are complete here: a caller may read them back from this point on
+  if (e == cudaSuccess && a->ev_attend_done)
+    e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(a->ev_attend_done), sm);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(ss, fork, 0);
   // side stream: selection for the next step
   if (e == cudaSuccess) e = mark(0, ss);

@@ -60,10 +60,11 @@ int main(void) {
          offsetof(asp_kv, page_table), offsetof(asp_kv, seq_lens));
   printf("asp_pred_cfg %zu %zu %zu %zu\n", sizeof(asp_pred_cfg), offsetof(asp_pred_cfg, windows), offsetof(asp_pred_cfg, lambda),
          offsetof(asp_pred_cfg, pool));
-  printf("asp_decode_args %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(asp_decode_args), offsetof(asp_decode_args, kv),
+  printf("asp_decode_args %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(asp_decode_args), offsetof(asp_decode_args, kv),
          offsetof(asp_decode_args, workspace_bytes), offsetof(asp_decode_args, s_main), offsetof(asp_decode_args, timing),
          offsetof(asp_decode_args, k_new), offsetof(asp_decode_args, quest_page), offsetof(asp_decode_args, pred_factor_cur),
-         offsetof(asp_decode_args, pred_factor_valid), offsetof(asp_decode_args, pred_factor_next));
+         offsetof(asp_decode_args, pred_factor_valid), offsetof(asp_decode_args, pred_factor_next),
+         offsetof(asp_decode_args, ev_attend_done));
   return 0;
 }
 '''
@@ -80,11 +81,11 @@ int main(void) {
     assert lines["asp_pred_cfg"] == [ctypes.sizeof(P), P.windows.offset, P.lam.offset, P.pool.offset]
     assert lines["asp_decode_args"] == [ctypes.sizeof(D), D.kv.offset, D.workspace_bytes.offset, D.s_main.offset,
                                         D.timing.offset, D.k_new.offset, D.quest_page.offset, D.pred_factor_cur.offset,
-                                        D.pred_factor_valid.offset, D.pred_factor_next.offset]
+                                        D.pred_factor_valid.offset, D.pred_factor_next.offset, D.ev_attend_done.offset]
 
 
 def test_version_and_status_strings(lib):
-    assert lib.asp_abi_version() == 4
+    assert lib.asp_abi_version() == 5
     assert L.status_string(L.ASP_OK) == "ok"
     assert "workspace" in L.status_string(L.ASP_ERR_WORKSPACE)
     assert L.status_string(99) == "unknown status"
