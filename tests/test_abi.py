@@ -278,6 +278,27 @@ def test_decode_step_and_wait_validation(lib):
     assert lib.asp_wait_selection(None, 10) == L.ASP_ERR_INVALID_ARG
 
 
+def test_decode_step_rejects_bad_factor_buffers(lib):
+    """The predictor-factor buffers are validated on the host before any launch:
+    8-byte aligned, and never the same buffer for this step and the next."""
+    B, Hkv, Hq, d, C = 2, 2, 4, 128, 64
+    kv = _kv(batch=B, n_kv_heads=Hkv, t_max=1024)
+    cfg = L.PredCfg(8, (4, 8), 1e-2)
+    a = L.AspDecodeArgs()
+    a.q_t, a.q_dtype, a.n_q_heads, a.qhist, a.ring_start = FAKE, L.ASP_BF16, Hq, FAKE, 0
+    a.pred, a.kv, a.C = ctypes.pointer(cfg.struct), ctypes.pointer(kv), C
+    a.idx_cur = a.count_cur = a.qpred = a.scores = a.idx_next = a.count_next = a.out = FAKE
+    a.workspace = 1 << 20   # 256-byte aligned, never dereferenced on the host
+    a.workspace_bytes = lib.asp_decode_workspace_bytes(B, Hq, Hkv, d, C, 0)
+    a.ev_fork = a.ev_sel_done = FAKE
+    a.pred_factor_cur, a.pred_factor_next = (1 << 21) + 4, 1 << 22      # misaligned
+    assert lib.asp_decode_step(ctypes.byref(a)) == L.ASP_ERR_INVALID_ARG
+    a.pred_factor_cur, a.pred_factor_next = 1 << 21, (1 << 22) + 2
+    assert lib.asp_decode_step(ctypes.byref(a)) == L.ASP_ERR_INVALID_ARG
+    a.pred_factor_cur = a.pred_factor_next = 1 << 21                   # the same buffer twice
+    assert lib.asp_decode_step(ctypes.byref(a)) == L.ASP_ERR_INVALID_ARG
+
+
 def test_wait_limit_check_validation(lib):
     assert lib.asp_check_wait_limit(8, None, None) == L.ASP_ERR_INVALID_ARG
     assert lib.asp_check_wait_limit(0, FAKE, None) == L.ASP_ERR_INVALID_ARG
